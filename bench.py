@@ -1,0 +1,519 @@
+"""Throughput bench of the paged-KV attention library on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                [--workload llama_decode|long_context|chat_trace|prefill_chunk]
+                [--block-size B] [--partition auto|none|<tokens>] [--no-e2e] [--no-cpu-baseline]
+
+A step is one pass of the hot path over one batch: map the step's new tokens
+to cache slots, write their K/V rows into the paged cache, then attend
+(single-pass decode, or split-KV + merge, or the chunked prefill). The default
+workload is the Llama-3-8B-shaped single-layer decode (64 sequences, 32 q / 8
+KV heads, head dim 128, block size 16, context lengths uniform in
+[512, 4096], fp16). Inputs are synthetic and resident in HBM before timing;
+the KV read per step (~0.6 GB) is larger than the 126 MB L2, so no flush is
+needed between steps.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own batch
+(weak scaling, no collective on the data path); the step time is the max
+over ranks and the value counts every rank's bytes.
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged-KV decode attention achieved HBM GB/s (% of peak) and seq-steps/s"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+WORKLOAD_DESC = {
+    "llama_decode": "Llama-3-8B-shaped single-layer paged decode fp16: batch 64, 32 q / 8 KV heads, head_dim 128, "
+                    "block_size 16, context_lens U[512,4096], pool 1.25x shuffled, one appended token per sequence",
+    "long_context": "long-context split-KV paged decode fp16: batch 4 x 100000 tokens, 32 q / 8 KV heads, "
+                    "head_dim 128, block_size 16, 512-token partitions + merge, q ~ N(0,2)",
+    "chat_trace": "chat-trace paged decode fp16: batch 256, lognormal context_lens (median 300, sigma 1, "
+                  "clipped [16,8192]), half sharing a 1024-token prefix, 32 q / 8 KV heads, head_dim 128",
+    "prefill_chunk": "chunked prefill bf16: batch 8, 512 causal query tokens after a paged context U[2048,8192], "
+                     "32 q / 8 KV heads, head_dim 128, block_size 16",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama_decode", choices=list(WORKLOAD_DESC))
+    ap.add_argument("--block-size", type=int, default=16)
+    ap.add_argument("--partition", default="auto")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the cpu_baseline sample")
+    a = ap.parse_args()
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+def make_workload(name, block_size, seed_offset=0, poison=None):
+    import workloads as W
+
+    if name == "llama_decode":
+        return W.llama_decode(block_size=block_size, poison=poison, seed=1 + seed_offset)
+    if name == "long_context":
+        return W.long_context(block_size=block_size, poison=poison, seed=2 + seed_offset)
+    if name == "chat_trace":
+        return W.chat_trace(block_size=block_size, poison=poison, seed=3 + seed_offset)
+    return W.prefill_chunk(block_size=block_size, poison=poison, seed=4 + seed_offset)
+
+
+def workload_bytes(batch):
+    """Algorithmic HBM bytes of one step (dict): the minimum a perfect kernel moves."""
+    import workloads as W
+
+    esz = batch.k_cache.element_size()
+    Hkv, D = batch.num_kv_heads, batch.head_dim
+    kv_logical = W.decode_kv_bytes(batch.context_lens.tolist(), Hkv, D, esz)
+    kv_unique = W.decode_kv_bytes(batch.context_lens.tolist(), Hkv, D, esz, batch.block_tables,
+                                  batch.block_size, unique=True)
+    q_out = 2 * batch.q.numel() * esz
+    nb = sum(W.blocks_for(int(L), batch.block_size) for L in batch.context_lens.tolist())
+    tables = nb * 4 + batch.num_seqs * 4
+    T = batch.new_seq.shape[0]
+    append = 2 * 2 * T * Hkv * D * esz + T * (8 + 8)  # new rows read + written, slots
+    return dict(kv_logical=kv_logical, kv_unique=kv_unique, q_out=q_out, tables=tables, append=append,
+                attend_logical=kv_logical + q_out + tables, attend_unique=kv_unique + q_out + tables)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", FALLBACK_HBM_GBS), d.get("bf16_tflops", FALLBACK_BF16_TFLOPS), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def kernel_traffic(kernel_key):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel_key)
+    if not d:
+        return None
+    if d.get("source_sha256") != source_hash(d.get("sources", [])):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+def source_hash(files):
+    h = hashlib.sha256()
+    for rel in files:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of SM clock and throttle reasons while the bench runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.flush()
+        self.f.seek(0)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.f.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_init(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    import torch
+
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, world):
+    import torch
+
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU side: the oracle on a bounded sample (cpu_baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(batch, n_seqs):
+    """A sub-batch of the first n_seqs sequences (same tables, same pool)."""
+    import copy
+
+    s = copy.copy(batch)
+    s.q = batch.q[:n_seqs]
+    s.block_tables = batch.block_tables[:n_seqs]
+    s.context_lens = batch.context_lens[:n_seqs]
+    keep = batch.new_seq < n_seqs
+    s.new_seq, s.new_pos = batch.new_seq[keep], batch.new_pos[keep]
+    s.k_new, s.v_new = batch.k_new[keep], batch.v_new[keep]
+    return s
+
+
+def time_oracle(batch_cpu, budget_s, prefill=False):
+    """Run the oracle step on growing samples until the budget is spent; returns (bytes_or_flops/s, info)."""
+    import oracle
+    import workloads as W
+
+    try:
+        from threadpoolctl import threadpool_info
+
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count() or 1
+    n = 1
+    done_units, spent, seqs_done, steps = 0.0, 0.0, 0, 0
+    while spent < budget_s and n <= batch_cpu.num_seqs:
+        s = oracle_sample(batch_cpu, n)
+        t0 = time.perf_counter()
+        if prefill:
+            oracle.step(s)
+            units = W.prefill_flops(s.context_lens.tolist(), s.chunk, s.num_q_heads, s.head_dim)
+        else:
+            oracle.step(s)
+            units = W.decode_kv_bytes(s.context_lens.tolist(), s.num_kv_heads, s.head_dim, s.k_cache.element_size())
+        dt = time.perf_counter() - t0
+        done_units += units
+        spent += dt
+        seqs_done += n
+        steps += 1
+        if dt * 2 < budget_s - spent:
+            n = min(batch_cpu.num_seqs, n * 2)
+    return done_units / spent, dict(cores=cores, seconds=round(spent, 2), seqs=seqs_done, samples=steps)
+
+
+def run_reference(args):
+    """--impl reference: the fp64 CPU oracle, as it stands, on a bounded sample of the workload."""
+    import torch  # noqa: F401
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    prefill = args.workload == "prefill_chunk"
+    batch = make_workload(args.workload, args.block_size)
+    per_step_budget = max(0.2, 100.0 / (args.steps + args.warmup))
+    # one sample size sized to the per-step budget
+    import oracle
+    import workloads as W
+
+    n = 1
+    while True:
+        s = oracle_sample(batch, n)
+        t0 = time.perf_counter()
+        oracle.step(s)
+        dt = time.perf_counter() - t0
+        if dt * 2 > per_step_budget or n >= batch.num_seqs:
+            break
+        n = min(batch.num_seqs, n * 2)
+    sample = oracle_sample(batch, n)
+    for _ in range(args.warmup):
+        oracle.step(sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.step(sample)
+    dt = time.perf_counter() - t0
+    if prefill:
+        units = W.prefill_flops(sample.context_lens.tolist(), sample.chunk, sample.num_q_heads, sample.head_dim)
+        value, unit = units * args.steps / dt / 1e12, "TFLOP/s"
+    else:
+        units = W.decode_kv_bytes(sample.context_lens.tolist(), sample.num_kv_heads, sample.head_dim,
+                                  sample.k_cache.element_size())
+        value, unit = units * args.steps / dt / 1e9, "GB/s"
+    try:
+        from threadpoolctl import threadpool_info
+
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count() or 1
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD_DESC[args.workload], "block_size": args.block_size},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": f"first {n} of {batch.num_seqs} sequences per step, fp64 numpy"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+# ---------------------------------------------------------------------------
+# GPU side
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+
+    world, rank, local = dist_init(args)
+    import paged_kv_cache_475_b200 as pa
+    from paged_kv_cache_475_b200.step import DecodeStep, PrefillStep
+
+    prefill = args.workload == "prefill_chunk"
+    batch_cpu = make_workload(args.workload, args.block_size, seed_offset=100 * rank)
+    batch = batch_cpu.to("cuda")
+    esz = batch.k_cache.element_size()
+    acct = workload_bytes(batch_cpu)
+    if prefill:
+        step = PrefillStep(batch.num_seqs, batch.chunk, batch.num_q_heads, batch.head_dim, batch.q.dtype,
+                           num_new_tokens=batch.new_seq.shape[0])
+        partition = None
+    else:
+        part = "auto" if args.partition == "auto" else (None if args.partition == "none" else int(args.partition))
+        step = DecodeStep(batch.num_seqs, batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
+                          int(batch_cpu.context_lens.max()), batch.q.dtype,
+                          num_new_tokens=batch.new_seq.shape[0], partition=part)
+        partition = step.partition
+    stream = torch.cuda.current_stream()
+    args_step = (batch.q, batch.k_new, batch.v_new, batch.k_cache, batch.v_cache, batch.block_tables,
+                 batch.context_lens, batch.new_seq, batch.new_pos, batch.scale)
+
+    # Split the step so that the dominant kernel can be timed on its own stream (the current one).
+    def run_step(ev=None):
+        B = batch.k_cache.shape[2]
+        pa.pa_slot_mapping(step.slot_mapping, batch.block_tables, batch.new_seq, batch.new_pos, B)
+        pa.pa_reshape_and_cache(batch.k_new, batch.v_new, batch.k_cache, batch.v_cache, step.slot_mapping)
+        if ev is not None:
+            ev[0].record(stream)
+        if prefill:
+            pa.pa_prefill_chunk(step.out, batch.q, batch.k_cache, batch.v_cache, batch.block_tables,
+                                batch.context_lens, batch.scale)
+        elif partition:
+            pa.pa_decode_splitkv(step.part_o, step.part_m, step.part_l, batch.q, batch.k_cache, batch.v_cache,
+                                 batch.block_tables, batch.context_lens, partition, batch.scale)
+        else:
+            pa.pa_decode(step.out, batch.q, batch.k_cache, batch.v_cache, batch.block_tables, batch.context_lens,
+                         batch.scale)
+        if ev is not None:
+            ev[1].record(stream)
+        if partition and not prefill:
+            pa.pa_merge(step.out, step.part_o, step.part_m, step.part_l, batch.context_lens, partition)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(args.warmup):
+        run_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(K):
+        run_step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+
+    ms_total = t_start.elapsed_time(t_end)
+    ms_total_max = max_over_ranks(ms_total, world)
+    ms_step = ms_total_max / K
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    flags = pa.pa_read_error_flags(clear=True)
+
+    hbm_peak, tf_peak, peak_src = measured_peaks()
+    if prefill:
+        import workloads as W
+
+        flops = W.prefill_flops(batch_cpu.context_lens.tolist(), batch.chunk, batch.num_q_heads, batch.head_dim)
+        units_rank = flops
+        value = sum_over_ranks(flops, world) / (ms_step / 1e3) / 1e12
+        unit = "TFLOP/s"
+        achieved = flops / (kern_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tf_peak, "unit": "TFLOP/s",
+                "frac": achieved / tf_peak, "traffic": kernel_traffic("prefill_chunk"),
+                "peak_source": f"{peak_src} bf16 burst (cuBLAS)", "kernel": "pa_prefill_chunk",
+                "kernel_ms": kern_ms}
+    else:
+        units_rank = acct["kv_logical"]
+        value = sum_over_ranks(units_rank, world) / (ms_step / 1e3) / 1e9
+        unit = "GB/s"
+        kname = "pa_decode_splitkv" if partition else "pa_decode"
+        attend_bytes = acct["attend_unique"]
+        achieved = attend_bytes / (kern_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": kernel_traffic(f"{kname}:{args.workload}:B{args.block_size}"),
+                "peak_source": f"{peak_src} HBM copy bandwidth", "kernel": kname, "kernel_ms": kern_ms,
+                "algorithmic_bytes_per_launch": attend_bytes}
+
+    # ---- end to end: host buffers in, result out, through the C ABI -----------
+    e2e = None
+    if not args.no_e2e:
+        host_in = [t.cpu().pin_memory() for t in (batch.q, batch.k_new, batch.v_new, batch.block_tables,
+                                                   batch.context_lens, batch.new_seq, batch.new_pos)]
+        dev_in = [batch.q, batch.k_new, batch.v_new, batch.block_tables, batch.context_lens, batch.new_seq,
+                  batch.new_pos]
+        host_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host_in)
+        d2h = host_out.numel() * host_out.element_size()
+
+        def e2e_step():
+            for h, d in zip(host_in, dev_in):
+                d.copy_(h, non_blocking=True)
+            step(*args_step)
+            host_out.copy_(step.out, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1), world) / K
+        e2e_val = sum_over_ranks(units_rank, world) / (ms_e2e / 1e3) / (1e12 if prefill else 1e9)
+        e2e = {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ms_e2e}
+
+    # ---- CPU baseline: the oracle on a bounded sample, rank 0 at N = 1 ---------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, info = time_oracle(batch_cpu, args.cpu_seconds, prefill)
+        cpu = {"value": v / (1e12 if prefill else 1e9), "unit": unit, "cores": info["cores"], "kind": "oracle",
+               "sample": f"fp64 numpy oracle step (append + attention) on the first 1,2,4,.. sequences of the "
+                         f"same batch; {info['seqs']} sequences over {info['samples']} runs in {info['seconds']} s"}
+
+    if rank == 0:
+        launches = step.launches_per_call * K
+        line = {
+            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": {"f16": "f16", "bf16": "bf16", "f32": "f32"}[batch_cpu.info["dtype"]], "data": "synthetic",
+            "config": {
+                "workload": WORKLOAD_DESC[args.workload], "num_seqs": batch.num_seqs, "block_size": batch.block_size,
+                "head_dim": batch.head_dim, "num_q_heads": batch.num_q_heads, "num_kv_heads": batch.num_kv_heads,
+                "partition": partition, "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
+                "kv_bytes_logical_per_rank": acct["kv_logical"], "kv_bytes_unique_per_rank": acct["kv_unique"],
+                "parallelism": f"dp{world} (independent batches per GPU)",
+            },
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "device_error_flags": flags,
+        }
+        if not prefill:
+            line["seq_steps_per_s"] = batch.num_seqs * world / (ms_step / 1e3)
+            line["pct_of_peak"] = 100.0 * value / (hbm_peak * world)
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -31,7 +31,8 @@ design notes):
    ceil(i/B), with the last block cut at token i.
  * prefill positions: context_lens counts the chunk; query i of a C-token
    chunk sits at position L-C+i and sees keys 0..L-C+i.
- * empty context: L = 0 gives a zero output row; an empty split partition has
+ * empty context: L = 0 gives a zero output row (so does a chunk query at a
+   negative position, L < C); an empty split partition has
    m = -inf, l = 0, o = 0 and drops out of the merge.
  * split partials: o_p is unnormalised, m_p is in natural-log units of the
    scaled score.
@@ -198,8 +199,6 @@ def attention(q, k_cache, v_cache, block_tables, context_lens, scale: float,
 
     for (b, kvh), items in sorted(wanted.items()):
         L = int(lens[b])
-        if L < C and L > 0:
-            raise ValueError("context_lens must count the chunk (L >= C)")
         K = gather_sequence(k_cache, bt[b], L, kvh)
         V = gather_sequence(v_cache, bt[b], L, kvh)
         qrows = np.stack([_as_f64(qq[b, i, h]) for (i, h) in items])

@@ -1,0 +1,89 @@
+"""Build libpa.so in-tree with nvcc for sm_100a (B200).
+
+python -m paged_kv_cache_475_b200.build [--force] [--verbose]
+
+Sources are compiled in parallel into _build/ (git-ignored) and linked into
+paged_kv_cache_475_b200/libpa.so. A rebuild happens only when a source or the
+public header is newer than the library.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import os
+import shutil
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+BUILD = os.path.join(ROOT, "_build")
+LIB = os.path.join(PKG, "libpa.so")
+HEADER = os.path.join(ROOT, "include", "pa.h")
+
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden",
+         "--expt-relaxed-constexpr", "-Xptxas", "-v"]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found: the CUDA toolkit is required to build libpa.so")
+
+
+def sources() -> list[str]:
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+
+
+def _stale() -> bool:
+    if not os.path.exists(LIB):
+        return True
+    t = os.path.getmtime(LIB)
+    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [HEADER]
+    return any(os.path.getmtime(d) > t for d in deps)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every CUDA source for sm_100a and link libpa.so; returns its path."""
+    if not force and not _stale():
+        return LIB
+    os.makedirs(BUILD, exist_ok=True)
+    cc = nvcc()
+    procs = []
+    objs = []
+    for src in sources():
+        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        log = obj + ".log"
+        objs.append(obj)
+        cmd = [cc, *ARCH, *FLAGS, "-c", src, "-o", obj]
+        f = open(log, "w")
+        procs.append((src, subprocess.Popen(cmd, stdout=f, stderr=subprocess.STDOUT), f, log))
+    failed = []
+    for src, pr, f, log in procs:
+        rc = pr.wait()
+        f.close()
+        text = open(log).read()
+        if verbose or rc:
+            sys.stderr.write(f"--- {os.path.basename(src)} (rc={rc})\n{text}\n")
+        if rc:
+            failed.append(src)
+    if failed:
+        raise RuntimeError(f"nvcc failed for: {', '.join(os.path.basename(s) for s in failed)}")
+    tmp = LIB + ".tmp"
+    link = [cc, *ARCH, "-shared", "-o", tmp, *objs]
+    r = subprocess.run(link, capture_output=True, text=True)
+    if r.returncode:
+        raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--verbose", action="store_true")
+    a = ap.parse_args()
+    print(build(force=a.force, verbose=a.verbose))

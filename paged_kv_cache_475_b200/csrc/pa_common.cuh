@@ -1,0 +1,169 @@
+// Shared device helpers for the paged-KV attention kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pa.h"
+
+namespace pa {
+
+// ---------------------------------------------------------------------------
+// Host-side helpers
+// ---------------------------------------------------------------------------
+
+// Device error word of the current device (lives in pa_api.cu).
+unsigned int* device_error_word();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool supported_block(int b) { return b == 8 || b == 16 || b == 32 || b == 64 || b == 128; }
+inline bool supported_head_dim(int d) { return d == 64 || d == 128; }
+inline bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+inline int dtype_bytes(pa_dtype dt) { return dt == PA_F32 ? 4 : 2; }
+
+inline int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Element types
+// ---------------------------------------------------------------------------
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static constexpr int kBytes = 4;
+  __device__ static inline float to_f(float x) { return x; }
+  __device__ static inline float from_f(float x) { return x; }
+};
+template <> struct Elem<__half> {
+  static constexpr int kBytes = 2;
+  __device__ static inline float to_f(__half x) { return __half2float(x); }
+  __device__ static inline __half from_f(float x) { return __float2half_rn(x); }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static constexpr int kBytes = 2;
+  __device__ static inline float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+  __device__ static inline __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+// Unpack a 16-byte chunk into floats (8 halves / 8 bf16 / 4 floats).
+__device__ inline void unpack16(const uint4& u, float* f, float) {
+  f[0] = __uint_as_float(u.x);
+  f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z);
+  f[3] = __uint_as_float(u.w);
+}
+__device__ inline void unpack16(const uint4& u, float* f, __half) {
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 v = __half22float2(h[i]);
+    f[2 * i] = v.x;
+    f[2 * i + 1] = v.y;
+  }
+}
+__device__ inline void unpack16(const uint4& u, float* f, __nv_bfloat16) {
+  // bf16 -> fp32 is exact: the bf16 bits are the high half of the float.
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// Unpack 2 x 32-bit words (8 bytes).
+__device__ inline void unpack8(const uint2& u, float* f, float) {
+  f[0] = __uint_as_float(u.x);
+  f[1] = __uint_as_float(u.y);
+}
+__device__ inline void unpack8(const uint2& u, float* f, __half) {
+  float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+  float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+  f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+}
+__device__ inline void unpack8(const uint2& u, float* f, __nv_bfloat16) {
+  f[0] = __uint_as_float(u.x << 16);
+  f[1] = __uint_as_float(u.x & 0xffff0000u);
+  f[2] = __uint_as_float(u.y << 16);
+  f[3] = __uint_as_float(u.y & 0xffff0000u);
+}
+// Unpack one 32-bit word (2 halves / 2 bf16 / 1 float).
+__device__ inline void unpack4(uint32_t u, float* f, float) { f[0] = __uint_as_float(u); }
+__device__ inline void unpack4(uint32_t u, float* f, __half) {
+  float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u));
+  f[0] = a.x; f[1] = a.y;
+}
+__device__ inline void unpack4(uint32_t u, float* f, __nv_bfloat16) {
+  f[0] = __uint_as_float(u << 16);
+  f[1] = __uint_as_float(u & 0xffff0000u);
+}
+
+// ---------------------------------------------------------------------------
+// Shared-memory barriers and bulk (TMA 1-D) copies, inline PTX
+// ---------------------------------------------------------------------------
+
+__device__ inline uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ inline void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ inline void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+// Bounded wait on a phase of an mbarrier. Returns false if the phase did not
+// complete within `limit` polls (the caller records PA_DEVERR_WAIT).
+__device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = (1u << 24)) {
+  const uint32_t a = smem_addr(bar);
+  for (uint32_t i = 0; i < limit; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+// Global -> shared bulk copy completing on an mbarrier (byte count, 16-byte
+// aligned addresses and size). L2 hint: evict-first (KV pages are streamed once).
+__device__ inline void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uint64_t* bar,
+                                uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+      ::"r"(smem_addr(dst_smem)), "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ inline uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ inline void set_error(unsigned int* err, unsigned int bit) {
+  if (err) atomicOr(err, bit);
+}
+
+// Packed fp32 FMA (sm_100): {a.x*b.x + c.x, a.y*b.y + c.y} in one instruction.
+__device__ inline float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+}  // namespace pa

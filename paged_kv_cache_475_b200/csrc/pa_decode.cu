@@ -1,0 +1,764 @@
+// Paged decode attention on CUDA cores: pa_decode, pa_decode_splitkv, pa_merge.
+//
+// What it computes: out = softmax(scale * q K^T) V for one query token per
+// sequence ("FlashAttention y PagedAttention", "Por qué la atención sale
+// cara"), with K/V read page by page through the block table (same page,
+// PagedAttention "Cómo funciona" step 5; "Cómo PagedAttention y RadixAttention
+// optimizan el manejo del KV cache en LLMs", step 2) and the softmax kept
+// online as a running max and running sum (FlashAttention "Cómo funciona").
+// Split-KV evaluates the per-partition sums of eq. (4) of "Flash Attention vs
+// Paged Attention" (算法原理) and pa_merge combines them.
+//
+// Design (B200, HBM-bound, no tensor cores):
+//  * one CTA per (sequence, KV head[, partition]); every K/V page is read once
+//    for all G = Hq/Hkv query heads of the group;
+//  * each warp owns a private ring of STAGES shared-memory stages; lane 0
+//    fills a stage with 1-D bulk copies (cp.async.bulk, TMA engine, no
+//    multicast) of one 16-token tile of K and of V straight out of the page
+//    that holds it, completing on the stage's mbarrier; block ids for the
+//    warp's next 32 tiles are prefetched into registers one chunk ahead;
+//  * scores: 8 (or 16) lanes split the head dim of one token, each lane keeps
+//    4 (or 8) tokens x G heads of partial dots in packed-fp32 FMAs, and a
+//    reduce-scatter over the lanes leaves every lane a few finished scores;
+//  * online softmax in the log2 domain (q pre-scaled by scale*log2(e)),
+//    probabilities through a 16 x G shared-memory slot, then P.V with each
+//    lane owning D/32 output dims for all G heads;
+//  * the warps' (m, l, o) states merge in shared memory at the end.
+#include "pa_common.cuh"
+
+namespace pa {
+
+constexpr int kTile = 16;              // tokens per pipeline stage
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <typename T, int D, int G>
+struct DecodeShape {
+  static constexpr int kEsz = static_cast<int>(sizeof(T));
+  static constexpr int kEpc = 16 / kEsz;                 // elements per 16-byte chunk
+  static constexpr int kRowChunks = D / kEpc;            // 16-byte chunks per row
+  static constexpr int kDGwant = (G >= 8) ? 16 : 8;
+  static constexpr int kDG = kDGwant < kRowChunks ? kDGwant : kRowChunks;  // lanes per token (dims split)
+  static constexpr int kTG = 32 / kDG;                   // token groups per warp
+  static constexpr int kTPL = kTile / kTG;               // tokens per lane, score phase
+  static constexpr int kCPL = kRowChunks / kDG;          // chunks per lane per token
+  static constexpr int kQPL = kCPL * kEpc;               // q values per lane per head
+  static constexpr int kNV = kTPL * G;                   // partial scores per lane
+  static constexpr int kNF = kNV >= kDG ? kNV / kDG : 1; // finished scores per lane
+  static constexpr int kDPL = D / 32;                    // output dims per lane, P.V phase
+  static constexpr int kTileBytes = kTile * D * kEsz;    // one K (or V) tile
+  static_assert(kCPL >= 1 && kQPL % 2 == 0, "head dim too small for the lane split");
+  static_assert(kDPL % 2 == 0, "D must be a multiple of 64");
+};
+
+struct DecodeParams {
+  void* out;                 // [N, Hq, D] (pa_decode)
+  float* part_o;             // [N, Hq, NP, D] (split)
+  float* part_m;             // [N, Hq, NP]
+  float* part_l;             // [N, Hq, NP]
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  unsigned int* err;
+  int max_blocks;
+  int num_seqs;
+  int num_q_heads;
+  int num_kv_heads;
+  int block_size;
+  int num_blocks;
+  int partition;             // tokens per partition; 0 = whole sequence
+  int num_parts;
+  float q_scale;             // scale * log2(e)
+};
+
+// Reduce-scatter of a[NV] over the kDG lanes of a token group (xor offsets
+// kDG/2 .. 1): at each level a lane keeps one half of its values and adds the
+// partner's copy of that half. Levels past a single value all-reduce.
+template <int NV, int OFF>
+struct ReduceScatter {
+  __device__ static inline void run(float* a, int lane) {
+    if constexpr (OFF >= 1) {
+      if constexpr (NV >= 2) {
+        constexpr int H = NV / 2;
+        const bool upper = (lane & OFF) != 0;
+#pragma unroll
+        for (int i = 0; i < H; ++i) {
+          const float send = upper ? a[i] : a[H + i];
+          const float keep = upper ? a[H + i] : a[i];
+          a[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
+        }
+        ReduceScatter<H, OFF / 2>::run(a, lane);
+      } else {
+        a[0] += __shfl_xor_sync(0xffffffffu, a[0], OFF);
+        ReduceScatter<1, OFF / 2>::run(a, lane);
+      }
+    }
+  }
+};
+
+// Index (into the original a[]) of a lane's first finished value.
+template <int NV, int DG>
+__device__ inline int scatter_base(int lane) {
+  int base = 0, n = NV;
+#pragma unroll
+  for (int off = DG / 2; off >= 1; off /= 2) {
+    if (n >= 2) {
+      n /= 2;
+      if (lane & off) base += n;
+    }
+  }
+  return base;
+}
+
+// Does xor offset `off` connect two lanes holding different tokens of the same
+// head (as opposed to different heads, or copies of the same value)?
+template <int NV, int DG, int TPL>
+__host__ __device__ constexpr bool same_head_offset(int off) {
+  if (off >= DG) return true;  // token-group bits
+  int n = NV;
+  for (int o = DG / 2; o >= 1; o /= 2) {
+    if (n >= 2) {
+      n /= 2;
+      if (o == off) return n < TPL;
+    } else if (o == off) {
+      return false;  // all-reduce level: both lanes hold the same value
+    }
+  }
+  return false;
+}
+
+template <int NV, int DG, int TPL, typename Op>
+__device__ inline float head_reduce(float v, Op op) {
+#pragma unroll
+  for (int off = 16; off >= 1; off /= 2)
+    if (same_head_offset<NV, DG, TPL>(off)) v = op(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
+
+// Lane (token group 0) that holds head g's first finished value.
+template <int NV, int DG, int TPL>
+__device__ inline int head_src_lane(int g) {
+  const int base = g * TPL;
+  int lane = 0, n = NV;
+#pragma unroll
+  for (int off = DG / 2; off >= 1; off /= 2) {
+    if (n >= 2) {
+      n /= 2;
+      if (base & n) lane |= off;
+    }
+  }
+  return lane;
+}
+
+struct MaxOp { __device__ float operator()(float a, float b) const { return fmaxf(a, b); } };
+struct SumOp { __device__ float operator()(float a, float b) const { return a + b; } };
+
+template <typename T, int D, int G, int NW, int STAGES>
+struct DecodeSmem {
+  using S = DecodeShape<T, D, G>;
+  static constexpr int kStageBytes = 2 * S::kTileBytes;
+  static constexpr int kRingBytes = NW * STAGES * kStageBytes;
+  static constexpr int kProbBytes = NW * kTile * G * 4;
+  static constexpr int kMergeBytes = NW * G * (D + 2) * 4;
+  static constexpr int kDataBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
+  static constexpr int kBarOff = kDataBytes + kProbBytes;
+  static constexpr int kValidOff = kBarOff + NW * STAGES * 8;
+  static constexpr int kTotal = kValidOff + NW * STAGES * 4;
+};
+
+template <typename T, int D, int G, int NW, int STAGES>
+__global__ void __launch_bounds__(NW * 32)
+decode_kernel(const DecodeParams p) {
+  using S = DecodeShape<T, D, G>;
+  using M = DecodeSmem<T, D, G, NW, STAGES>;
+  extern __shared__ __align__(128) unsigned char smem[];
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int part = blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
+  const bool split = p.partition > 0;
+
+  // ---- context range of this CTA -------------------------------------------
+  int L = p.context_lens[b];
+  if (L < 0 || L > p.max_blocks * p.block_size) {
+    if (threadIdx.x == 0) set_error(p.err, PA_DEVERR_CONTEXT);
+    L = L < 0 ? 0 : p.max_blocks * p.block_size;
+  }
+  if (split && part == p.num_parts - 1 && L > p.num_parts * p.partition && threadIdx.x == 0)
+    set_error(p.err, PA_DEVERR_CONTEXT);
+  const int t_begin = split ? part * p.partition : 0;
+  int t_end = split ? min(L, t_begin + p.partition) : L;
+  if (t_end < t_begin) t_end = t_begin;
+  const int n_tiles = (t_end - t_begin + kTile - 1) / kTile;
+  const int my_tiles = warp < n_tiles ? (n_tiles - warp + NW - 1) / NW : 0;
+
+  unsigned char* ring = smem + warp * STAGES * M::kStageBytes;
+  float* prob = reinterpret_cast<float*>(smem + M::kDataBytes) + warp * kTile * G;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + M::kBarOff) + warp * STAGES;
+  int* stage_valid = reinterpret_cast<int*>(smem + M::kValidOff) + warp * STAGES;
+
+  if (lane == 0) {
+    for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  const T* kc = static_cast<const T*>(p.k_cache);
+  const T* vc = static_cast<const T*>(p.v_cache);
+  const int32_t* bt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
+  const int B = p.block_size;
+  const int n_seq_blocks = (L + B - 1) / B;
+  const uint64_t policy = l2_evict_first_policy();
+
+  // Block ids of this warp's tiles k = 32*c + lane (two ids per tile when B = 8).
+  auto load_ids = [&](int chunk, int& id0, int& id1) {
+    const int k = chunk * 32 + lane;
+    id0 = -1;
+    id1 = -1;
+    if (k < my_tiles) {
+      const int t0 = t_begin + (warp + NW * k) * kTile;
+      const int j = t0 / B;
+      id0 = bt[j];
+      if (B < kTile && j + 1 < n_seq_blocks && t0 + B < t_end) id1 = bt[j + 1];
+    }
+  };
+  int cur0, cur1, nxt0, nxt1;
+  load_ids(0, cur0, cur1);
+  load_ids(1, nxt0, nxt1);
+  int ids_chunk = 0;
+
+  // Issue the copies of tile k into stage k % STAGES (all lanes call; lane 0 copies).
+  auto issue = [&](int k) {
+    const int chunk = k >> 5;
+    if (chunk != ids_chunk) {  // advance the prefetched id window
+      cur0 = nxt0;
+      cur1 = nxt1;
+      ids_chunk = chunk;
+      load_ids(chunk + 1, nxt0, nxt1);
+    }
+    const int id0 = __shfl_sync(0xffffffffu, cur0, k & 31);
+    const int id1 = __shfl_sync(0xffffffffu, cur1, k & 31);
+    if (lane == 0) {
+      const int s = k % STAGES;
+      const int t0 = t_begin + (warp + NW * k) * kTile;
+      const int nvalid = min(kTile, t_end - t0);
+      unsigned char* kdst = ring + s * M::kStageBytes;
+      unsigned char* vdst = kdst + S::kTileBytes;
+      // Validate every block id before any copy; a bad id skips the tile.
+      bool ok;
+      const bool second = B < kTile && nvalid > B;
+      if (B >= kTile) {
+        ok = id0 >= 0 && id0 < p.num_blocks;
+      } else {
+        ok = id0 >= 0 && id0 < p.num_blocks && (!second || (id1 >= 0 && id1 < p.num_blocks));
+      }
+      // The stage's valid-token count is written before the arrive (release),
+      // so the lanes that acquire the completed phase see it.
+      stage_valid[s] = ok ? nvalid : 0;
+      if (!ok) {
+        set_error(p.err, PA_DEVERR_BLOCK_ID);
+        mbar_arrive_expect_tx(&bars[s], 0);
+      } else if (B >= kTile) {
+        const int64_t off = ((static_cast<int64_t>(id0) * p.num_kv_heads + kvh) * B + (t0 % B)) * D;
+        mbar_arrive_expect_tx(&bars[s], 2u * S::kTileBytes);
+        bulk_g2s(kdst, kc + off, S::kTileBytes, &bars[s], policy);
+        bulk_g2s(vdst, vc + off, S::kTileBytes, &bars[s], policy);
+      } else {  // B == 8: two half tiles, the second only if it holds a valid token
+        const uint32_t half = S::kTileBytes / 2;
+        mbar_arrive_expect_tx(&bars[s], (second ? 2u : 1u) * 2u * half);
+        const int64_t off0 = (static_cast<int64_t>(id0) * p.num_kv_heads + kvh) * B * D;
+        bulk_g2s(kdst, kc + off0, half, &bars[s], policy);
+        bulk_g2s(vdst, vc + off0, half, &bars[s], policy);
+        if (second) {
+          const int64_t off1 = (static_cast<int64_t>(id1) * p.num_kv_heads + kvh) * B * D;
+          bulk_g2s(kdst + half, kc + off1, half, &bars[s], policy);
+          bulk_g2s(vdst + half, vc + off1, half, &bars[s], policy);
+        }
+      }
+    }
+  };
+
+  // ---- q for this lane: G heads x kQPL dims, pre-scaled ----------------------
+  const int dg = lane % S::kDG;
+  const int tg = lane / S::kDG;
+  float2 q2[G][S::kQPL / 2];
+  {
+    const T* qb = static_cast<const T*>(p.q) + (static_cast<int64_t>(b) * p.num_q_heads + kvh * G) * D;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+#pragma unroll
+      for (int c = 0; c < S::kCPL; ++c) {
+        const int ci = c * S::kDG + dg;
+        const uint4 u = *reinterpret_cast<const uint4*>(qb + g * D + ci * S::kEpc);
+        float f[S::kEpc];
+        unpack16(u, f, T());
+#pragma unroll
+        for (int e = 0; e < S::kEpc; e += 2)
+          q2[g][(c * S::kEpc + e) / 2] = make_float2(f[e] * p.q_scale, f[e + 1] * p.q_scale);
+      }
+    }
+  }
+
+  // ---- running state ---------------------------------------------------------
+  float m_run[G];
+  float2 acc[G][S::kDPL / 2];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    m_run[g] = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < S::kDPL / 2; ++j) acc[g][j] = make_float2(0.f, 0.f);
+  }
+  float l_part = 0.f;  // partial sum of this lane's own head, own tokens
+  const int base_idx = scatter_base<S::kNV, S::kDG>(lane);
+  const int my_head = base_idx / S::kTPL;
+
+  // ---- pipeline --------------------------------------------------------------
+  const int prologue = my_tiles < STAGES ? my_tiles : STAGES;
+  for (int k = 0; k < prologue; ++k) issue(k);
+  __syncwarp();
+
+  bool aborted = false;
+  int k = 0;
+  for (; k < my_tiles; ++k) {
+    const int s = k % STAGES;
+    if (!mbar_wait(&bars[s], (k / STAGES) & 1)) {
+      if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
+      aborted = true;
+      break;
+    }
+    const int nvalid = stage_valid[s];
+    const unsigned char* ktile = ring + s * M::kStageBytes;
+    const unsigned char* vtile = ktile + S::kTileBytes;
+
+    if (nvalid > 0) {
+      // -- scores: partial dots over this lane's dims for its kTPL tokens --
+      float a[S::kNV];
+      {
+        float2 part2[G][S::kTPL];
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int i = 0; i < S::kTPL; ++i) part2[g][i] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < S::kTPL; ++i) {
+          const int t = tg + S::kTG * i;
+#pragma unroll
+          for (int c = 0; c < S::kCPL; ++c) {
+            const int ci = c * S::kDG + dg;
+            const uint4 u = *reinterpret_cast<const uint4*>(ktile + (t * S::kRowChunks + ci) * 16);
+            float f[S::kEpc];
+            unpack16(u, f, T());
+#pragma unroll
+            for (int e = 0; e < S::kEpc; e += 2) {
+              const float2 kv = make_float2(f[e], f[e + 1]);
+#pragma unroll
+              for (int g = 0; g < G; ++g) part2[g][i] = ffma2(q2[g][(c * S::kEpc + e) / 2], kv, part2[g][i]);
+            }
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+          for (int i = 0; i < S::kTPL; ++i) a[g * S::kTPL + i] = part2[g][i].x + part2[g][i].y;
+      }
+      ReduceScatter<S::kNV, S::kDG / 2>::run(a, lane);
+
+      // -- mask and tile max per head --
+      float vmax = -INFINITY;
+#pragma unroll
+      for (int f = 0; f < S::kNF; ++f) {
+        const int idx = base_idx + f;
+        const int t = tg + S::kTG * (idx % S::kTPL);
+        if (t >= nvalid) a[f] = -INFINITY;
+        vmax = fmaxf(vmax, a[f]);
+      }
+      vmax = head_reduce<S::kNV, S::kDG, S::kTPL>(vmax, MaxOp());
+      float alpha[G], m_use[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float tmax = __shfl_sync(0xffffffffu, vmax, head_src_lane<S::kNV, S::kDG, S::kTPL>(g));
+        const float m_new = fmaxf(m_run[g], tmax);
+        m_use[g] = m_new == -INFINITY ? 0.f : m_new;
+        alpha[g] = exp2f(m_run[g] - m_use[g]);  // exp2(-inf) = 0 on the first tile
+        m_run[g] = m_new;
+      }
+      // -- probabilities of this lane's scores into the tile's prob slot --
+      float psum = 0.f;
+#pragma unroll
+      for (int f = 0; f < S::kNF; ++f) {
+        const int idx = base_idx + f;
+        const int t = tg + S::kTG * (idx % S::kTPL);
+        float mh = m_use[0];
+#pragma unroll
+        for (int g = 1; g < G; ++g) mh = (my_head == g) ? m_use[g] : mh;
+        const float pr = exp2f(a[f] - mh);
+        psum += pr;
+        prob[t * G + my_head] = pr;
+      }
+      {
+        float ah = alpha[0];
+#pragma unroll
+        for (int g = 1; g < G; ++g) ah = (my_head == g) ? alpha[g] : ah;
+        l_part = l_part * ah + psum;
+      }
+      __syncwarp();
+
+      // -- P.V: this lane's kDPL output dims for all G heads --
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int j = 0; j < S::kDPL / 2; ++j) {
+          acc[g][j].x *= alpha[g];
+          acc[g][j].y *= alpha[g];
+        }
+      auto pv_token = [&](int t) {
+        float vf[S::kDPL];
+        const unsigned char* vrow = vtile + (t * D + lane * S::kDPL) * S::kEsz;
+        if constexpr (S::kDPL * S::kEsz == 16) {
+          unpack16(*reinterpret_cast<const uint4*>(vrow), vf, T());
+        } else if constexpr (S::kDPL * S::kEsz == 8) {
+          unpack8(*reinterpret_cast<const uint2*>(vrow), vf, T());
+        } else {
+          unpack4(*reinterpret_cast<const uint32_t*>(vrow), vf, T());
+        }
+        float pg[G];
+        if constexpr (G % 4 == 0) {
+#pragma unroll
+          for (int g = 0; g < G; g += 4) {
+            const float4 p4 = *reinterpret_cast<const float4*>(prob + t * G + g);
+            pg[g] = p4.x; pg[g + 1] = p4.y; pg[g + 2] = p4.z; pg[g + 3] = p4.w;
+          }
+        } else if constexpr (G == 2) {
+          const float2 p2 = *reinterpret_cast<const float2*>(prob + t * G);
+          pg[0] = p2.x; pg[1] = p2.y;
+        } else {
+          pg[0] = prob[t];
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float2 pp = make_float2(pg[g], pg[g]);
+#pragma unroll
+          for (int j = 0; j < S::kDPL / 2; ++j)
+            acc[g][j] = ffma2(pp, make_float2(vf[2 * j], vf[2 * j + 1]), acc[g][j]);
+        }
+      };
+      if (nvalid == kTile) {
+#pragma unroll
+        for (int t = 0; t < kTile; ++t) pv_token(t);
+      } else {
+        for (int t = 0; t < nvalid; ++t) pv_token(t);
+      }
+    }
+    __syncwarp();
+    if (k + STAGES < my_tiles) issue(k + STAGES);
+  }
+
+  if (aborted) {
+    // Let this warp's copies still in flight land before the CTA exits.
+    const int issued = my_tiles < k + STAGES ? my_tiles : k + STAGES;
+    for (int kk = k; kk < issued; ++kk) mbar_wait(&bars[kk % STAGES], (kk / STAGES) & 1, 1u << 20);
+  }
+
+  // ---- per-warp finish: l for every head -------------------------------------
+  const float l_head = head_reduce<S::kNV, S::kDG, S::kTPL>(l_part, SumOp());
+  float l_run[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) l_run[g] = __shfl_sync(0xffffffffu, l_head, head_src_lane<S::kNV, S::kDG, S::kTPL>(g));
+
+  __syncthreads();  // every warp is done with its ring: reuse it for the merge
+  float* mo = reinterpret_cast<float*>(smem);                   // [NW][G][D]
+  float* mm = mo + NW * G * D;                                   // [NW][G]
+  float* ml = mm + NW * G;                                       // [NW][G]
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+#pragma unroll
+    for (int j = 0; j < S::kDPL / 2; ++j)
+      *reinterpret_cast<float2*>(mo + (warp * G + g) * D + lane * S::kDPL + 2 * j) = acc[g][j];
+    if (lane == 0) {
+      mm[warp * G + g] = m_run[g];
+      ml[warp * G + g] = l_run[g];
+    }
+  }
+  __syncthreads();
+
+  for (int i = threadIdx.x; i < G * D; i += NW * 32) {
+    const int g = i / D, d = i % D;
+    float Mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) Mx = fmaxf(Mx, mm[w * G + g]);
+    float o = 0.f, l = 0.f;
+    if (Mx != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float mw = mm[w * G + g];
+        if (mw == -INFINITY) continue;
+        const float sc = exp2f(mw - Mx);
+        o += sc * mo[(w * G + g) * D + d];
+        l += sc * ml[w * G + g];
+      }
+    }
+    const int h = kvh * G + g;
+    if (split) {
+      const int64_t row = (static_cast<int64_t>(b) * p.num_q_heads + h) * p.num_parts + part;
+      p.part_o[row * D + d] = o;
+      if (d == 0) {
+        p.part_m[row] = Mx == -INFINITY ? -INFINITY : Mx * kLn2;
+        p.part_l[row] = l;
+      }
+    } else {
+      T* out = static_cast<T*>(p.out) + (static_cast<int64_t>(b) * p.num_q_heads + h) * D;
+      out[d] = Elem<T>::from_f(l > 0.f ? o / l : 0.f);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Merge of split-KV partials: one CTA of MW warps per (sequence, head); warp
+// w folds partitions w, w+MW, ... online, then the warps combine in smem.
+// ---------------------------------------------------------------------------
+template <typename T, int D, int MW>
+__global__ void __launch_bounds__(MW * 32)
+merge_kernel(T* __restrict__ out, const float* __restrict__ part_o, const float* __restrict__ part_m,
+             const float* __restrict__ part_l, const int32_t* __restrict__ context_lens, int num_q_heads,
+             int partition, int num_parts) {
+  constexpr int DPL = D / 32;
+  __shared__ float s_o[MW][D];
+  __shared__ float s_m[MW], s_l[MW];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int row = blockIdx.x;  // b * Hq + h
+  const int b = row / num_q_heads;
+  int L = context_lens[b];
+  L = L < 0 ? 0 : L;
+  int np = (L + partition - 1) / partition;
+  np = np > num_parts ? num_parts : np;
+  const float* po = part_o + static_cast<int64_t>(row) * num_parts * D;
+  const float* pm = part_m + static_cast<int64_t>(row) * num_parts;
+  const float* pl = part_l + static_cast<int64_t>(row) * num_parts;
+
+  float m_run = -INFINITY, l_run = 0.f;
+  float o[DPL];
+#pragma unroll
+  for (int j = 0; j < DPL; ++j) o[j] = 0.f;
+  for (int pp = warp; pp < np; pp += MW) {
+    const float l = pl[pp];
+    if (!(l > 0.f)) continue;
+    const float m = pm[pp];
+    float v[DPL];
+    if constexpr (DPL == 4) {
+      const float4 x = *reinterpret_cast<const float4*>(po + pp * D + lane * 4);
+      v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    } else {
+      const float2 x = *reinterpret_cast<const float2*>(po + pp * D + lane * 2);
+      v[0] = x.x; v[1] = x.y;
+    }
+    const float m_new = fmaxf(m_run, m);
+    const float a = expf(m_run - m_new);  // 0 on the first live partition
+    const float w = expf(m - m_new);
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) o[j] = o[j] * a + w * v[j];
+    l_run = l_run * a + w * l;
+    m_run = m_new;
+  }
+#pragma unroll
+  for (int j = 0; j < DPL; ++j) s_o[warp][lane * DPL + j] = o[j];
+  if (lane == 0) {
+    s_m[warp] = m_run;
+    s_l[warp] = l_run;
+  }
+  __syncthreads();
+  for (int d = threadIdx.x; d < D; d += MW * 32) {
+    float Mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < MW; ++w) Mx = fmaxf(Mx, s_m[w]);
+    float num = 0.f, den = 0.f;
+    if (Mx != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < MW; ++w) {
+        if (s_m[w] == -INFINITY) continue;
+        const float sc = expf(s_m[w] - Mx);
+        num += sc * s_o[w][d];
+        den += sc * s_l[w];
+      }
+    }
+    out[static_cast<int64_t>(row) * D + d] = Elem<T>::from_f(den > 0.f ? num / den : 0.f);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+constexpr int kDecodeWarps = 4;
+constexpr int kDecodeStages = 4;
+
+template <typename T, int D, int G>
+int launch_decode(const DecodeParams& prm, int grid_x, cudaStream_t stream) {
+  constexpr int NW = kDecodeWarps;
+  constexpr int ST = (DecodeShape<T, D, G>::kTileBytes >= 8192) ? 2 : kDecodeStages;
+  using M = DecodeSmem<T, D, G, NW, ST>;
+  auto kern = decode_kernel<T, D, G, NW, ST>;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, M::kTotal) != cudaSuccess)
+      return PA_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  dim3 grid(grid_x, prm.num_kv_heads, prm.num_seqs);
+  kern<<<grid, NW * 32, M::kTotal, stream>>>(prm);
+  return launch_status();
+}
+
+template <typename T, int D>
+int dispatch_group(const DecodeParams& prm, int G, int grid_x, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_decode<T, D, 1>(prm, grid_x, s);
+    case 2: return launch_decode<T, D, 2>(prm, grid_x, s);
+    case 4: return launch_decode<T, D, 4>(prm, grid_x, s);
+    case 8: return launch_decode<T, D, 8>(prm, grid_x, s);
+  }
+  return PA_ERR_UNSUPPORTED;
+}
+
+template <typename T>
+int dispatch_dim(const DecodeParams& prm, int D, int G, int grid_x, cudaStream_t s) {
+  if (D == 64) return dispatch_group<T, 64>(prm, G, grid_x, s);
+  if (D == 128) return dispatch_group<T, 128>(prm, G, grid_x, s);
+  return PA_ERR_UNSUPPORTED;
+}
+
+int run_decode(DecodeParams prm, int D, float scale, pa_dtype dt, int grid_x, cudaStream_t s) {
+  const int G = prm.num_q_heads / prm.num_kv_heads;
+  prm.q_scale = scale * kLog2e;
+  prm.err = device_error_word();
+  switch (dt) {
+    case PA_F32: return dispatch_dim<float>(prm, D, G, grid_x, s);
+    case PA_F16: return dispatch_dim<__half>(prm, D, G, grid_x, s);
+    case PA_BF16: return dispatch_dim<__nv_bfloat16>(prm, D, G, grid_x, s);
+  }
+  return PA_ERR_DTYPE;
+}
+
+int check_decode_args(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      int max_blocks, const int32_t* context_lens, int num_seqs, int num_q_heads,
+                      int num_kv_heads, int head_dim, int block_size, int num_blocks, pa_dtype dt) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks < 0 || max_blocks < 0)
+    return PA_ERR_SHAPE;
+  if (dt != PA_F32 && dt != PA_F16 && dt != PA_BF16) return PA_ERR_DTYPE;
+  if (num_q_heads % num_kv_heads) return PA_ERR_SHAPE;
+  if (!supported_head_dim(head_dim) || !supported_block(block_size) ||
+      !supported_group(num_q_heads / num_kv_heads))
+    return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_ALIGN;
+  return PA_OK;
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" PA_API int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                const int32_t* block_tables, int max_blocks_per_seq,
+                                const int32_t* context_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+                                int head_dim, int block_size, int num_blocks, float scale, pa_dtype dtype,
+                                void* stream) {
+  int st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                             num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, dtype);
+  if (st != PA_OK || num_seqs == 0) return st;
+  if (!out) return PA_ERR_NULL;
+  if (num_seqs > 65535) return PA_ERR_SHAPE;
+  DecodeParams prm{};
+  prm.out = out;
+  prm.q = q;
+  prm.k_cache = k_cache;
+  prm.v_cache = v_cache;
+  prm.block_tables = block_tables;
+  prm.context_lens = context_lens;
+  prm.max_blocks = max_blocks_per_seq;
+  prm.num_seqs = num_seqs;
+  prm.num_q_heads = num_q_heads;
+  prm.num_kv_heads = num_kv_heads;
+  prm.block_size = block_size;
+  prm.num_blocks = num_blocks;
+  prm.partition = 0;
+  prm.num_parts = 1;
+  return run_decode(prm, head_dim, scale, dtype, 1, (cudaStream_t)stream);
+}
+
+extern "C" PA_API int pa_decode_splitkv(float* part_o, float* part_m, float* part_l, const void* q,
+                                        const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                                        int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                                        int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                        int num_blocks, int partition_size, int num_partitions, float scale,
+                                        pa_dtype dtype, void* stream) {
+  int st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                             num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, dtype);
+  if (st != PA_OK || num_seqs == 0) return st;
+  if (!part_o || !part_m || !part_l) return PA_ERR_NULL;
+  if (!aligned16(part_o)) return PA_ERR_ALIGN;
+  if (partition_size <= 0 || partition_size % kTile || num_partitions <= 0) return PA_ERR_WORKSPACE;
+  if (num_seqs > 65535 || num_partitions > (1 << 30)) return PA_ERR_SHAPE;
+  DecodeParams prm{};
+  prm.part_o = part_o;
+  prm.part_m = part_m;
+  prm.part_l = part_l;
+  prm.q = q;
+  prm.k_cache = k_cache;
+  prm.v_cache = v_cache;
+  prm.block_tables = block_tables;
+  prm.context_lens = context_lens;
+  prm.max_blocks = max_blocks_per_seq;
+  prm.num_seqs = num_seqs;
+  prm.num_q_heads = num_q_heads;
+  prm.num_kv_heads = num_kv_heads;
+  prm.block_size = block_size;
+  prm.num_blocks = num_blocks;
+  prm.partition = partition_size;
+  prm.num_parts = num_partitions;
+  return run_decode(prm, head_dim, scale, dtype, num_partitions, (cudaStream_t)stream);
+}
+
+namespace pa {
+template <typename T>
+int launch_merge(void* out, const float* po, const float* pm, const float* pl, const int32_t* lens, int rows,
+                 int Hq, int D, int partition, int np, cudaStream_t s) {
+  constexpr int MW = 4;
+  if (D == 64)
+    merge_kernel<T, 64, MW><<<rows, MW * 32, 0, s>>>(static_cast<T*>(out), po, pm, pl, lens, Hq, partition, np);
+  else if (D == 128)
+    merge_kernel<T, 128, MW><<<rows, MW * 32, 0, s>>>(static_cast<T*>(out), po, pm, pl, lens, Hq, partition, np);
+  else
+    return PA_ERR_UNSUPPORTED;
+  return launch_status();
+}
+}  // namespace pa
+
+extern "C" PA_API int pa_merge(void* out, const float* part_o, const float* part_m, const float* part_l,
+                               const int32_t* context_lens, int num_seqs, int num_q_heads, int head_dim,
+                               int partition_size, int num_partitions, pa_dtype dtype, void* stream) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_partitions <= 0) return PA_ERR_SHAPE;
+  if (!supported_head_dim(head_dim)) return PA_ERR_UNSUPPORTED;
+  if (partition_size <= 0) return PA_ERR_WORKSPACE;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !part_o || !part_m || !part_l || !context_lens) return PA_ERR_NULL;
+  if (!aligned16(part_o)) return PA_ERR_ALIGN;
+  const int64_t rows = static_cast<int64_t>(num_seqs) * num_q_heads;
+  if (rows > 0x7fffffff) return PA_ERR_SHAPE;
+  cudaStream_t s = (cudaStream_t)stream;
+  switch (dtype) {
+    case PA_F32: return launch_merge<float>(out, part_o, part_m, part_l, context_lens, (int)rows, num_q_heads,
+                                            head_dim, partition_size, num_partitions, s);
+    case PA_F16: return launch_merge<__half>(out, part_o, part_m, part_l, context_lens, (int)rows, num_q_heads,
+                                             head_dim, partition_size, num_partitions, s);
+    case PA_BF16: return launch_merge<__nv_bfloat16>(out, part_o, part_m, part_l, context_lens, (int)rows,
+                                                     num_q_heads, head_dim, partition_size, num_partitions, s);
+  }
+  return PA_ERR_DTYPE;
+}

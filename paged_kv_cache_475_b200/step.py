@@ -1,0 +1,99 @@
+"""One decode or prefill step through the C ABI, with preallocated buffers.
+
+A step is what a serving loop runs per layer: map the step's new tokens to
+cache slots (pa_slot_mapping), write their K/V rows (pa_reshape_and_cache),
+then attend (pa_decode, or pa_decode_splitkv + pa_merge for long or few
+contexts, or pa_prefill_chunk). Buffers are allocated once in the
+constructor, so a step allocates nothing and can be replayed from a CUDA
+graph. Every call goes to libpa.so; nothing here computes.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (pa_decode, pa_decode_splitkv, pa_merge, pa_prefill_chunk, pa_reshape_and_cache,
+               pa_slot_mapping, pa_splitkv_num_partitions)
+
+NUM_SMS_B200 = 148
+
+
+def choose_partition(num_seqs: int, num_kv_heads: int, max_context_len: int,
+                     num_sms: int = NUM_SMS_B200) -> int | None:
+    """Split-KV partition size for a decode batch, or None for the single-pass kernel.
+
+    Single pass reads every page once and needs no workspace; it is chosen
+    when there are enough (sequence, KV head) CTAs to fill the GPU and no
+    context is very long. Otherwise the context is cut into 512-token
+    partitions so that the work spreads over all SMs.
+    """
+    ctas = num_seqs * num_kv_heads
+    if ctas >= 3 * num_sms and max_context_len <= 8192:
+        return None
+    return 512
+
+
+class DecodeStep:
+    """Append one token per sequence, then decode-attend over the paged cache."""
+
+    def __init__(self, num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                 max_context_len: int, dtype: torch.dtype, num_new_tokens: int | None = None,
+                 partition: int | None | str = "auto", device="cuda"):
+        self.N, self.Hq, self.D = num_seqs, num_q_heads, head_dim
+        if partition == "auto":
+            partition = choose_partition(num_seqs, num_kv_heads, max_context_len)
+        self.partition = partition
+        T = num_seqs if num_new_tokens is None else num_new_tokens
+        self.slot_mapping = torch.empty(T, dtype=torch.int64, device=device)
+        self.out = torch.empty((num_seqs, num_q_heads, head_dim), dtype=dtype, device=device)
+        if partition:
+            self.num_parts = pa_splitkv_num_partitions(max_context_len, partition)
+            self.part_o = torch.empty((num_seqs, num_q_heads, self.num_parts, head_dim), dtype=torch.float32,
+                                      device=device)
+            self.part_m = torch.empty((num_seqs, num_q_heads, self.num_parts), dtype=torch.float32, device=device)
+            self.part_l = torch.empty_like(self.part_m)
+        self.launches_per_call = 4 if partition else 3
+
+    def __call__(self, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, new_seq, new_pos,
+                 scale: float, stream=None):
+        B = k_cache.shape[2]
+        pa_slot_mapping(self.slot_mapping, block_tables, new_seq, new_pos, B, stream)
+        pa_reshape_and_cache(k_new, v_new, k_cache, v_cache, self.slot_mapping, stream)
+        if self.partition:
+            pa_decode_splitkv(self.part_o, self.part_m, self.part_l, q, k_cache, v_cache, block_tables,
+                              context_lens, self.partition, scale, stream)
+            pa_merge(self.out, self.part_o, self.part_m, self.part_l, context_lens, self.partition, stream)
+        else:
+            pa_decode(self.out, q, k_cache, v_cache, block_tables, context_lens, scale, stream)
+        return self.out
+
+
+class PrefillStep:
+    """Append a C-token chunk per sequence, then causal chunk attention over the paged cache."""
+
+    def __init__(self, num_seqs: int, chunk: int, num_q_heads: int, head_dim: int, dtype: torch.dtype,
+                 num_new_tokens: int | None = None, device="cuda"):
+        T = num_seqs * chunk if num_new_tokens is None else num_new_tokens
+        self.slot_mapping = torch.empty(T, dtype=torch.int64, device=device)
+        self.out = torch.empty((num_seqs, chunk, num_q_heads, head_dim), dtype=dtype, device=device)
+        self.launches_per_call = 3
+
+    def __call__(self, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, new_seq, new_pos,
+                 scale: float, stream=None):
+        B = k_cache.shape[2]
+        pa_slot_mapping(self.slot_mapping, block_tables, new_seq, new_pos, B, stream)
+        pa_reshape_and_cache(k_new, v_new, k_cache, v_cache, self.slot_mapping, stream)
+        pa_prefill_chunk(self.out, q, k_cache, v_cache, block_tables, context_lens, scale, stream)
+        return self.out
+
+
+def run_batch(batch, partition: int | None | str = "auto"):
+    """Run one step of a workloads.PagedBatch that lives on the GPU; returns the output tensor."""
+    if batch.chunk == 1:
+        step = DecodeStep(batch.num_seqs, batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
+                          int(batch.context_lens.max().item()) if batch.num_seqs else 1, batch.q.dtype,
+                          num_new_tokens=batch.new_seq.shape[0], partition=partition)
+    else:
+        step = PrefillStep(batch.num_seqs, batch.chunk, batch.num_q_heads, batch.head_dim, batch.q.dtype,
+                           num_new_tokens=batch.new_seq.shape[0])
+    return step(batch.q, batch.k_new, batch.v_new, batch.k_cache, batch.v_cache, batch.block_tables,
+                batch.context_lens, batch.new_seq, batch.new_pos, batch.scale)

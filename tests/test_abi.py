@@ -1,0 +1,92 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU, exports every declared symbol,
+and rejects bad arguments on the host (no kernel is launched by these calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_475_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = B.build()
+    return ctypes.CDLL(path)
+
+
+def declared_symbols():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"PA_API\s+[\w\s\*]+?\b(pa_\w+)\s*\(", text)
+    return names
+
+
+def test_header_declares_entry_points():
+    names = set(declared_symbols())
+    for n in ("pa_reshape_and_cache", "pa_decode", "pa_decode_splitkv", "pa_merge", "pa_prefill_chunk",
+              "pa_slot_mapping", "pa_read_error_flags", "pa_status_string"):
+        assert n in names
+
+
+def test_exports_every_declared_symbol(lib):
+    missing = [n for n in declared_symbols() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_version(lib):
+    lib.pa_status_string.restype = ctypes.c_char_p
+    assert lib.pa_status_string(0) == b"PA_OK"
+    for code in range(-7, 0):
+        assert lib.pa_status_string(code).startswith(b"PA_ERR")
+    assert lib.pa_version() >= 100
+
+
+def test_num_partitions(lib):
+    f = lib.pa_splitkv_num_partitions
+    assert f(100000, 512) == 196
+    assert f(512, 512) == 1
+    assert f(513, 512) == 2
+    assert f(0, 512) == 1
+    assert f(10, 0) == 0
+
+
+def _decode_args(**kw):
+    fake = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    a = dict(out=fake, q=fake, k=fake, v=fake, bt=fake, mb=4, lens=fake, N=2, Hq=8, Hkv=2, D=128, B=16, P=10,
+             scale=ctypes.c_float(0.1), dt=1, stream=None)
+    a.update(kw)
+    return list(a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=96), -4), (dict(B=24), -4), (dict(Hq=6, Hkv=4), -2), (dict(Hq=48, Hkv=2), -4),
+    (dict(dt=7), -3), (dict(q=None), -1), (dict(N=-1), -2), (dict(q=ctypes.c_void_p(24)), -7),
+])
+def test_decode_rejects_bad_args_on_host(lib, kw, code):
+    assert lib.pa_decode(*_decode_args(**kw)) == code
+
+
+def test_splitkv_rejects_bad_partition(lib):
+    fake = ctypes.c_void_p(16)
+    args = [fake, fake, fake, fake, fake, fake, fake, 4, fake, 2, 8, 2, 128, 16, 10, 24, 3,
+            ctypes.c_float(0.1), 1, None]
+    assert lib.pa_decode_splitkv(*args) == -5  # partition not a multiple of 16
+    args[15] = 512
+    args[16] = 0
+    assert lib.pa_decode_splitkv(*args) == -5  # no partitions
+
+
+def test_prefill_rejects_f32(lib):
+    fake = ctypes.c_void_p(16)
+    args = [fake, fake, fake, fake, fake, 4, fake, 2, 8, 8, 2, 128, 16, 10, ctypes.c_float(0.1), 0, None]
+    assert lib.pa_prefill_chunk(*args) == -3
+
+
+def test_zero_sized_calls_are_noops(lib):
+    assert lib.pa_slot_mapping(None, None, 0, None, None, 0, 0, 16, None) == 0
+    assert lib.pa_reshape_and_cache(None, None, None, None, None, 0, 10, 8, 128, 16, 1, None) == 0

@@ -1,0 +1,66 @@
+"""Parity at the full workload sizes, in the launch configuration bench.py times.
+
+The Llama-3-8B-shaped decode and the chat trace (every block size of the
+sweep) are compared in full; the 100k-token split-KV decode and the chunked
+prefill on sampled output rows, which the oracle computes one by one. Pools
+are NaN-poisoned outside what each sequence may read.
+"""
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests.gpu_common import assert_close, gather_rows, require_gpu, run_gpu, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    require_gpu()
+
+
+@pytest.fixture(scope="module")
+def llama():
+    b = W.llama_decode()
+    ref, *_ = oracle.step(b)
+    return b, ref
+
+
+@pytest.mark.parametrize("partition", ["auto", None, 512])
+def test_llama_decode_full(llama, partition):
+    b, ref = llama
+    out, _, flags = run_gpu(b, partition=partition)
+    assert flags == 0
+    assert_close(out, ref, "f16", f"llama decode partition={partition}")
+
+
+def test_long_context_sampled():
+    b = W.long_context()
+    out, _, flags = run_gpu(b, partition="auto")
+    assert flags == 0
+    rows = [(s, 0, h) for s in range(b.num_seqs) for h in (0, 3, 4, 17, 31)]
+    kc, vc = oracle.reshape_and_cache(b.k_new, b.v_new, b.k_cache, b.v_cache,
+                                      oracle.slot_mapping(b.block_tables, b.new_seq, b.new_pos, b.block_size))
+    ref = oracle.attention(b.q, kc, vc, b.block_tables, b.context_lens, b.scale, rows=rows)
+    assert_close(gather_rows(out, rows, 1), ref, "f16", "100k split-KV")
+
+
+@pytest.mark.parametrize("B", [8, 16, 32, 64, 128])
+def test_chat_trace_full(B):
+    b = W.chat_trace(block_size=B)
+    ref, *_ = oracle.step(b)
+    out, _, flags = run_gpu(b, partition="auto")
+    assert flags == 0
+    assert_close(out, ref, "f16", f"chat trace B={B}")
+
+
+def test_prefill_chunk_sampled():
+    b = W.prefill_chunk()
+    out, _, flags = run_gpu(b)
+    assert flags == 0
+    rows = sample_rows(b, 96)
+    kc, vc = oracle.reshape_and_cache(b.k_new, b.v_new, b.k_cache, b.v_cache,
+                                      oracle.slot_mapping(b.block_tables, b.new_seq, b.new_pos, b.block_size))
+    ref = oracle.attention(b.q, kc, vc, b.block_tables, b.context_lens, b.scale, rows=rows)
+    assert_close(gather_rows(out, rows, b.chunk), ref, "bf16", "prefill chunk")

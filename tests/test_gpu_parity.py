@@ -1,0 +1,285 @@
+"""CUDA path vs the fp64 oracle on the same seeded inputs (element by element).
+
+Cache write and slot indices: bit-exact. Attention outputs: max-abs <= 1e-2 and
+mean-abs <= 1e-3 for fp16/bf16, max-abs <= 1e-5 for fp32. Invariants that the
+pages fix (block relabelling, shared blocks) must hold bit for bit on the GPU,
+since the kernels' reduction order does not depend on physical block ids.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests.gpu_common import (assert_close, permute_pool, require_gpu, run_gpu, small_batch)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    require_gpu()
+
+
+# ---------------------------------------------------------------------------
+# Cache write
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B", [8, 16, 32, 64, 128])
+def test_slot_mapping_and_cache_write_bit_exact(B):
+    import paged_kv_cache_475_b200 as pa
+    b = small_batch(seed=100 + B, B=B, chunk=5, lens=(5, 9, 40, 129, 300), dtype="bf16")
+    g = b.to("cuda")
+    # padding tokens (seq -1) mixed in
+    seq = torch.cat([g.new_seq, torch.full((3,), -1, dtype=torch.int32, device="cuda")])
+    pos = torch.cat([g.new_pos, torch.zeros(3, dtype=torch.int32, device="cuda")])
+    slots = torch.empty(seq.shape[0], dtype=torch.int64, device="cuda")
+    pa.pa_slot_mapping(slots, g.block_tables, seq, pos, B)
+    ref_slots = oracle.slot_mapping(b.block_tables, seq.cpu(), pos.cpu(), B)
+    assert slots.cpu().numpy().tolist() == ref_slots.tolist()
+    kn = torch.cat([g.k_new, torch.zeros((3,) + tuple(g.k_new.shape[1:]), dtype=g.k_new.dtype, device="cuda")])
+    vn = torch.cat([g.v_new, torch.zeros_like(kn[-3:])])
+    pa.pa_reshape_and_cache(kn, vn, g.k_cache, g.v_cache, slots)
+    torch.cuda.synchronize()
+    kc, vc = oracle.reshape_and_cache(kn.cpu(), vn.cpu(), b.k_cache, b.v_cache, ref_slots)
+    assert torch.equal(g.k_cache.cpu().view(torch.int16), kc.view(torch.int16))
+    assert torch.equal(g.v_cache.cpu().view(torch.int16), vc.view(torch.int16))
+    assert pa.pa_read_error_flags() == 0
+
+
+def test_cache_write_f32_and_out_of_pool_slot():
+    import paged_kv_cache_475_b200 as pa
+    b = W.tiny_fp32()
+    g = b.to("cuda")
+    slots = torch.tensor([3, -1, 16 * 16 + 5, 17], dtype=torch.int64, device="cuda")  # third is past the pool
+    kn = torch.randn(4, 1, 64, device="cuda")
+    vn = torch.randn(4, 1, 64, device="cuda")
+    pa.pa_reshape_and_cache(kn, vn, g.k_cache, g.v_cache, slots)
+    flags = pa.pa_read_error_flags()
+    assert flags & pa.DEVERR_SLOT
+    ok = torch.tensor([3, -1, -1, 17])
+    kc, vc = oracle.reshape_and_cache(kn.cpu(), vn.cpu(), b.k_cache, b.v_cache, ok)
+    assert torch.equal(g.k_cache.cpu().view(torch.int32), kc.view(torch.int32))
+    assert torch.equal(g.v_cache.cpu().view(torch.int32), vc.view(torch.int32))
+
+
+# ---------------------------------------------------------------------------
+# Decode
+# ---------------------------------------------------------------------------
+
+def test_tiny_fp32_decode():
+    b = W.tiny_fp32()
+    ref, *_ = oracle.step(b)
+    for part in (None, 16, 32):
+        out, _, flags = run_gpu(b, partition=part)
+        assert flags == 0
+        assert_close(out, ref, "f32", f"tiny fp32 partition={part}")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("B", [8, 16, 32, 64, 128])
+def test_decode_grid_f16(D, G, B):
+    b = small_batch(seed=D * 1000 + G * 100 + B, D=D, G=G, B=B)
+    ref, *_ = oracle.step(b)
+    out, _, flags = run_gpu(b, partition=None)
+    assert flags == 0
+    assert_close(out, ref, "f16", f"D={D} G={G} B={B}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B", [8, 16, 128])
+@pytest.mark.parametrize("D,G", [(128, 4), (64, 2), (128, 8)])
+def test_decode_other_dtypes(dtype, B, D, G):
+    b = small_batch(seed=7 + B + D + G, dtype=dtype, D=D, G=G, B=B)
+    ref, *_ = oracle.step(b)
+    out, _, flags = run_gpu(b, partition=None)
+    assert flags == 0
+    assert_close(out, ref, dtype, f"{dtype} D={D} G={G} B={B}")
+
+
+@pytest.mark.parametrize("poison", [float("nan"), 65504.0, -65504.0])
+def test_decode_poisoned_pool_is_never_read(poison):
+    b = small_batch(seed=31, poison=poison, lens=(1, 2, 31, 33, 250))
+    ref, *_ = oracle.step(b)
+    for part in (None, 64):
+        out, _, flags = run_gpu(b, partition=part)
+        assert flags == 0
+        assert_close(out, ref, "f16", f"poison={poison} partition={part}")
+
+
+def test_decode_peaky_softmax():
+    b = small_batch(seed=41, q_std=2.0 ** 0.5 * 3, lens=(64, 513, 1000))
+    ref, *_ = oracle.step(b)
+    out, _, _ = run_gpu(b, partition=None)
+    assert_close(out, ref, "f16", "peaky")
+
+
+def test_decode_empty_and_single_token():
+    import paged_kv_cache_475_b200 as pa
+    b = small_batch(seed=51, lens=(1, 1, 5))
+    g = b.to("cuda")
+    g.context_lens[2] = 0  # an empty context: zero row, nothing read
+    from paged_kv_cache_475_b200.step import run_batch
+    out = run_batch(g, partition=None)
+    torch.cuda.synchronize()
+    assert not out[2].any()
+    # one visible token: the softmax weight is exactly 1, so out equals V[0] bit for bit
+    for s in (0, 1):
+        blk = int(b.block_tables[s, 0])
+        for h in range(b.num_q_heads):
+            v0 = b.v_new[s, h // (b.num_q_heads // b.num_kv_heads)]
+            assert torch.equal(out[s, h].cpu(), v0)
+    assert pa.pa_read_error_flags() == 0
+
+
+def test_decode_block_permutation_bit_identical():
+    b = small_batch(seed=61, lens=(3, 100, 517, 999))
+    out1, _, _ = run_gpu(b, partition=None)
+    out2, _, _ = run_gpu(permute_pool(b), partition=None)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    out3, _, _ = run_gpu(b, partition=64)
+    out4, _, _ = run_gpu(permute_pool(b, seed=9), partition=64)
+    assert torch.equal(out3.view(torch.int16), out4.view(torch.int16))
+
+
+def test_decode_shared_blocks_equal_private_copies():
+    b = small_batch(seed=71, B=16, lens=(300, 200, 129, 50), shared_prefix_tokens=128, shared_group=3)
+    out1, _, _ = run_gpu(b, partition=None)
+    # give sequences 1 and 2 private copies of the 8 shared blocks
+    b2 = b.to("cpu")
+    b2.k_cache, b2.v_cache, b2.block_tables = b.k_cache.clone(), b.v_cache.clone(), b.block_tables.clone()
+    used = set(b.block_tables[b.block_tables >= 0].tolist())
+    spare = [i for i in range(b.k_cache.shape[0]) if i not in used]
+    assert len(spare) >= 16
+    for s in (1, 2):
+        for j in range(8):
+            src, dst = int(b.block_tables[s, j]), spare.pop()
+            b2.k_cache[dst], b2.v_cache[dst] = b.k_cache[src], b.v_cache[src]
+            b2.block_tables[s, j] = dst
+    out2, _, _ = run_gpu(b2, partition=None)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+def test_decode_bad_block_id_sets_flag_without_fault():
+    import paged_kv_cache_475_b200 as pa
+    b = small_batch(seed=81, lens=(40, 70, 90))
+    ref, *_ = oracle.step(b)
+    bad = b.to("cpu")
+    bad.block_tables = b.block_tables.clone()
+    bad.block_tables[0, 1] = b.k_cache.shape[0] + 5  # outside the pool
+    for part in (None, 32):
+        g = bad.to("cuda")
+        pa.pa_read_error_flags(clear=True)
+        # the append only touches each sequence's last block, not block 1 of sequence 0
+        from paged_kv_cache_475_b200.step import run_batch
+        out = run_batch(g, partition=part).cpu()
+        flags = pa.pa_read_error_flags(clear=True)
+        assert flags & pa.DEVERR_BLOCK_ID
+        assert_close(out[1:], ref[1:], "f16", "unaffected sequences")
+
+
+# ---------------------------------------------------------------------------
+# Split-KV partials and merge
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("partition", [16, 64, 512, 4096])
+@pytest.mark.parametrize("B", [8, 16, 128])
+def test_splitkv_partials_and_merge(partition, B):
+    import paged_kv_cache_475_b200 as pa
+    b = small_batch(seed=91 + partition + B, B=B, lens=(1, 16, 17, 511, 512, 513, 1400))
+    out, g, flags = run_gpu(b, partition=partition)
+    assert flags == 0
+    ref, kc, vc, _ = oracle.step(b)
+    assert_close(out, ref, "f16", f"merged partition={partition} B={B}")
+    # the partials themselves
+    NP = pa.pa_splitkv_num_partitions(int(b.context_lens.max()), partition)
+    po, pm, pl = pa.splitkv_buffers(b.num_seqs, b.num_q_heads, b.head_dim, NP)
+    pa.pa_decode_splitkv(po, pm, pl, g.q, g.k_cache, g.v_cache, g.block_tables, g.context_lens, partition, b.scale)
+    torch.cuda.synchronize()
+    o_ref, m_ref, l_ref = oracle.splitkv_partials(b.q, kc, vc, b.block_tables, b.context_lens, b.scale,
+                                                  partition, NP)
+    pm, pl, po = pm.cpu().double().numpy(), pl.cpu().double().numpy(), po.cpu().double().numpy()
+    live = l_ref > 0
+    assert (pl[~live] == 0).all() and np.isneginf(pm[~live]).all() and (po[~live] == 0).all()
+    assert np.abs(pm[live] - m_ref[live]).max() < 1e-4
+    assert (np.abs(pl[live] - l_ref[live]) / l_ref[live]).max() < 1e-4
+    on = po[live] / pl[live][:, None]
+    on_ref = o_ref[live] / l_ref[live][:, None]
+    assert np.abs(on - on_ref).max() < 1e-3
+
+
+def test_merge_skips_partitions_past_context():
+    import paged_kv_cache_475_b200 as pa
+    N, Hq, NP, D = 3, 4, 5, 128
+    gen = torch.Generator().manual_seed(3)
+    o = torch.randn(N, Hq, NP, D, generator=gen)
+    m = torch.randn(N, Hq, NP, generator=gen)
+    l = torch.rand(N, Hq, NP, generator=gen) + 0.5
+    lens = torch.tensor([64, 200, 0], dtype=torch.int32)  # partition 64 -> 1, 4, 0 partitions
+    live_o, live_m, live_l = o.clone().double().numpy(), m.clone().double().numpy(), l.clone().double().numpy()
+    for b_, npb in enumerate([1, 4, 0]):
+        live_l[b_, :, npb:] = 0.0
+    ref = oracle.merge(live_o, live_m, live_l)
+    out = torch.empty(N, Hq, D, dtype=torch.float32, device="cuda")
+    pa.pa_merge(out, o.cuda(), m.cuda(), l.cuda(), lens.cuda(), 64)
+    torch.cuda.synchronize()
+    assert np.abs(out.cpu().double().numpy() - ref).max() < 1e-5
+    assert not out[2].any()
+
+
+# ---------------------------------------------------------------------------
+# Chunked prefill
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_prefill_grid(D, G, dtype):
+    b = small_batch(seed=D + G * 10 + len(dtype), dtype=dtype, D=D, G=G, B=16, chunk=37,
+                    lens=(37, 38, 100, 229, 500))
+    ref, *_ = oracle.step(b)
+    out, _, flags = run_gpu(b)
+    assert flags == 0
+    assert_close(out, ref, dtype, f"prefill D={D} G={G} {dtype}")
+
+
+@pytest.mark.parametrize("B", [8, 32, 64, 128])
+@pytest.mark.parametrize("C", [1, 16, 64, 130])
+def test_prefill_blocks_and_chunks(B, C):
+    b = small_batch(seed=B * 7 + C, dtype="bf16", D=128, G=4, B=B, chunk=C, lens=(C, C + 1, C + 63, C + 300))
+    ref, *_ = oracle.step(b)
+    out, _, flags = run_gpu(b)
+    assert flags == 0
+    assert_close(out, ref, "bf16", f"prefill B={B} C={C}")
+
+
+def test_prefill_permutation_bit_identical():
+    b = small_batch(seed=5, dtype="bf16", chunk=40, lens=(40, 90, 333))
+    out1, _, _ = run_gpu(b)
+    out2, _, _ = run_gpu(permute_pool(b))
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+def test_prefill_short_context_rows_are_zero():
+    """L < C: the first C - L queries sit at negative positions and see nothing."""
+    import paged_kv_cache_475_b200 as pa
+    from paged_kv_cache_475_b200.step import PrefillStep
+    b = small_batch(seed=6, dtype="bf16", chunk=20, lens=(20, 40))
+    g = b.to("cuda")
+    step = PrefillStep(b.num_seqs, b.chunk, b.num_q_heads, b.head_dim, g.q.dtype,
+                       num_new_tokens=g.new_seq.shape[0])
+    step(g.q, g.k_new, g.v_new, g.k_cache, g.v_cache, g.block_tables, g.context_lens, g.new_seq, g.new_pos,
+         b.scale)
+    lens = g.context_lens.clone()
+    lens[0] = 12  # only 12 keys visible for sequence 0: queries 0..7 see nothing
+    out = torch.empty_like(g.q)
+    pa.pa_prefill_chunk(out, g.q, g.k_cache, g.v_cache, g.block_tables, lens, b.scale)
+    torch.cuda.synchronize()
+    assert not out[0, :8].any()
+    _, kc, vc, _ = oracle.step(b)  # the oracle's own append
+    rows = [(0, i, h) for i in range(20) for h in range(b.num_q_heads)]
+    ref = oracle.attention(b.q, kc, vc, b.block_tables, lens.cpu(), b.scale, rows=rows)
+    assert not ref[: 8 * b.num_q_heads].any()
+    got = torch.stack([out[0, i, h].cpu() for (_, i, h) in rows])
+    assert_close(got, ref, "bf16", "short context")
