@@ -46,19 +46,22 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every CUDA source for sm_100a and link libpa.so; returns its path."""
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, defines=(), lib: str = LIB, objdir: str = BUILD) -> str:
+    """Compile every CUDA source for sm_100a and link libpa.so; returns its path.
+
+    defines: extra -D macros (tuning variants), written to `lib` with objects in `objdir`.
+    """
+    if not force and lib == LIB and not _stale():
         return LIB
-    os.makedirs(BUILD, exist_ok=True)
+    os.makedirs(objdir, exist_ok=True)
     cc = nvcc()
     procs = []
     objs = []
     for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
         log = obj + ".log"
         objs.append(obj)
-        cmd = [cc, *ARCH, *FLAGS, "-c", src, "-o", obj]
+        cmd = [cc, *ARCH, *FLAGS, *[f"-D{d}" for d in defines], "-c", src, "-o", obj]
         f = open(log, "w")
         procs.append((src, subprocess.Popen(cmd, stdout=f, stderr=subprocess.STDOUT), f, log))
     failed = []
@@ -72,13 +75,13 @@ def build(force: bool = False, verbose: bool = False) -> str:
             failed.append(src)
     if failed:
         raise RuntimeError(f"nvcc failed for: {', '.join(os.path.basename(s) for s in failed)}")
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     link = [cc, *ARCH, "-shared", "-o", tmp, *objs]
     r = subprocess.run(link, capture_output=True, text=True)
     if r.returncode:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":

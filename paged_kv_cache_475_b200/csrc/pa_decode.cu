@@ -70,8 +70,31 @@ struct DecodeParams {
   int num_blocks;
   int partition;             // tokens per partition; 0 = whole sequence
   int num_parts;
+  int longest_first;         // map CTA z-index r to the r-th longest sequence
   float q_scale;             // scale * log2(e)
 };
+
+// Sequence whose context is the r-th longest (ties by index). CTAs are
+// dispatched in z order, so the longest contexts start first and short ones
+// fill the tail (greedy longest-processing-time scheduling). O(N^2 / threads)
+// compares per CTA, used for small batches only.
+__device__ inline int longest_first_seq(const int32_t* lens, int n, int r, int* slot) {
+  if (threadIdx.x == 0) *slot = r;
+  __syncthreads();
+  for (int j = threadIdx.x; j < n; j += blockDim.x) {
+    const int Lj = lens[j];
+    int rank = 0;
+    for (int i = 0; i < n; ++i) {
+      const int Li = lens[i];
+      rank += (Li > Lj) || (Li == Lj && i < j);
+    }
+    if (rank == r) *slot = j;
+  }
+  __syncthreads();
+  const int b = *slot;
+  __syncthreads();
+  return b;
+}
 
 // Reduce-scatter of a[NV] over the kDG lanes of a token group (xor offsets
 // kDG/2 .. 1): at each level a lane keeps one half of its values and adds the
@@ -165,11 +188,15 @@ struct DecodeSmem {
   static constexpr int kDataBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
   static constexpr int kBarOff = kDataBytes + kProbBytes;
   static constexpr int kValidOff = kBarOff + NW * STAGES * 8;
-  static constexpr int kTotal = kValidOff + NW * STAGES * 4;
+  static constexpr int kTotal = kValidOff + NW * STAGES * 4 + 16;
 };
 
+#ifndef PA_DECODE_MINB
+#define PA_DECODE_MINB 1
+#endif
+
 template <typename T, int D, int G, int NW, int STAGES>
-__global__ void __launch_bounds__(NW * 32)
+__global__ void __launch_bounds__(NW * 32, PA_DECODE_MINB)
 decode_kernel(const DecodeParams p) {
   using S = DecodeShape<T, D, G>;
   using M = DecodeSmem<T, D, G, NW, STAGES>;
@@ -179,8 +206,11 @@ decode_kernel(const DecodeParams p) {
   const int warp = threadIdx.x >> 5;
   const int part = blockIdx.x;
   const int kvh = blockIdx.y;
-  const int b = blockIdx.z;
   const bool split = p.partition > 0;
+  const int b = p.longest_first
+                    ? longest_first_seq(p.context_lens, p.num_seqs, blockIdx.z,
+                                        reinterpret_cast<int*>(smem + M::kValidOff + NW * STAGES * 4))
+                    : static_cast<int>(blockIdx.z);
 
   // ---- context range of this CTA -------------------------------------------
   int L = p.context_lens[b];
@@ -517,9 +547,29 @@ decode_kernel(const DecodeParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// Merge of split-KV partials: one CTA of MW warps per (sequence, head); warp
-// w folds partitions w, w+MW, ... online, then the warps combine in smem.
+// Merge of split-KV partials: one CTA of MW warps per (sequence, head).
+// Pass 1 (all threads): M = max m_p and Lsum = sum exp(m_p - M) l_p over the
+// live partitions. Pass 2: warp w accumulates exp(m_p - M) o_p for partitions
+// w, w+MW, ...; the loads of successive partitions are independent, so many
+// are in flight at once. The warps' sums meet in shared memory.
 // ---------------------------------------------------------------------------
+template <int MW>
+__device__ inline float block_reduce(float v, float* red, bool is_max) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off >= 1; off /= 2) {
+    const float o = __shfl_xor_sync(0xffffffffu, v, off);
+    v = is_max ? fmaxf(v, o) : v + o;
+  }
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int w = 1; w < MW; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
+  __syncthreads();
+  return r;
+}
+
 template <typename T, int D, int MW>
 __global__ void __launch_bounds__(MW * 32)
 merge_kernel(T* __restrict__ out, const float* __restrict__ part_o, const float* __restrict__ part_m,
@@ -527,7 +577,7 @@ merge_kernel(T* __restrict__ out, const float* __restrict__ part_o, const float*
              int partition, int num_parts) {
   constexpr int DPL = D / 32;
   __shared__ float s_o[MW][D];
-  __shared__ float s_m[MW], s_l[MW];
+  __shared__ float red[MW];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int row = blockIdx.x;  // b * Hq + h
   const int b = row / num_q_heads;
@@ -539,51 +589,45 @@ merge_kernel(T* __restrict__ out, const float* __restrict__ part_o, const float*
   const float* pm = part_m + static_cast<int64_t>(row) * num_parts;
   const float* pl = part_l + static_cast<int64_t>(row) * num_parts;
 
-  float m_run = -INFINITY, l_run = 0.f;
+  float mloc = -INFINITY;
+  for (int pp = threadIdx.x; pp < np; pp += MW * 32)
+    if (pl[pp] > 0.f) mloc = fmaxf(mloc, pm[pp]);
+  const float M = block_reduce<MW>(mloc, red, true);
+  float dloc = 0.f;
+  if (M != -INFINITY)
+    for (int pp = threadIdx.x; pp < np; pp += MW * 32) {
+      const float l = pl[pp];
+      dloc += l > 0.f ? expf(pm[pp] - M) * l : 0.f;
+    }
+  const float den = block_reduce<MW>(dloc, red, false);
+
   float o[DPL];
 #pragma unroll
   for (int j = 0; j < DPL; ++j) o[j] = 0.f;
-  for (int pp = warp; pp < np; pp += MW) {
-    const float l = pl[pp];
-    if (!(l > 0.f)) continue;
-    const float m = pm[pp];
-    float v[DPL];
-    if constexpr (DPL == 4) {
-      const float4 x = *reinterpret_cast<const float4*>(po + pp * D + lane * 4);
-      v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-    } else {
-      const float2 x = *reinterpret_cast<const float2*>(po + pp * D + lane * 2);
-      v[0] = x.x; v[1] = x.y;
-    }
-    const float m_new = fmaxf(m_run, m);
-    const float a = expf(m_run - m_new);  // 0 on the first live partition
-    const float w = expf(m - m_new);
+  if (M != -INFINITY) {
+#pragma unroll 4
+    for (int pp = warp; pp < np; pp += MW) {
+      const float l = pl[pp];
+      const float w = l > 0.f ? expf(pm[pp] - M) : 0.f;
+      float v[DPL];
+      if constexpr (DPL == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(po + static_cast<int64_t>(pp) * D + lane * 4);
+        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2*>(po + static_cast<int64_t>(pp) * D + lane * 2);
+        v[0] = x.x; v[1] = x.y;
+      }
 #pragma unroll
-    for (int j = 0; j < DPL; ++j) o[j] = o[j] * a + w * v[j];
-    l_run = l_run * a + w * l;
-    m_run = m_new;
+      for (int j = 0; j < DPL; ++j) o[j] += l > 0.f ? w * v[j] : 0.f;
+    }
   }
 #pragma unroll
   for (int j = 0; j < DPL; ++j) s_o[warp][lane * DPL + j] = o[j];
-  if (lane == 0) {
-    s_m[warp] = m_run;
-    s_l[warp] = l_run;
-  }
   __syncthreads();
   for (int d = threadIdx.x; d < D; d += MW * 32) {
-    float Mx = -INFINITY;
+    float num = 0.f;
 #pragma unroll
-    for (int w = 0; w < MW; ++w) Mx = fmaxf(Mx, s_m[w]);
-    float num = 0.f, den = 0.f;
-    if (Mx != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < MW; ++w) {
-        if (s_m[w] == -INFINITY) continue;
-        const float sc = expf(s_m[w] - Mx);
-        num += sc * s_o[w][d];
-        den += sc * s_l[w];
-      }
-    }
+    for (int w = 0; w < MW; ++w) num += s_o[w][d];
     out[static_cast<int64_t>(row) * D + d] = Elem<T>::from_f(den > 0.f ? num / den : 0.f);
   }
 }
@@ -592,13 +636,22 @@ merge_kernel(T* __restrict__ out, const float* __restrict__ part_o, const float*
 // Host side
 // ---------------------------------------------------------------------------
 
-constexpr int kDecodeWarps = 4;
-constexpr int kDecodeStages = 4;
+#ifndef PA_DECODE_WARPS
+#define PA_DECODE_WARPS 4
+#endif
+#ifndef PA_DECODE_STAGES
+#define PA_DECODE_STAGES 2
+#endif
+#ifndef PA_DECODE_LPT_MAX_SEQS
+#define PA_DECODE_LPT_MAX_SEQS 256
+#endif
+constexpr int kDecodeWarps = PA_DECODE_WARPS;
+constexpr int kDecodeStages = PA_DECODE_STAGES;
 
 template <typename T, int D, int G>
 int launch_decode(const DecodeParams& prm, int grid_x, cudaStream_t stream) {
   constexpr int NW = kDecodeWarps;
-  constexpr int ST = (DecodeShape<T, D, G>::kTileBytes >= 8192) ? 2 : kDecodeStages;
+  constexpr int ST = (DecodeShape<T, D, G>::kTileBytes >= 8192 && kDecodeStages > 2) ? 2 : kDecodeStages;
   using M = DecodeSmem<T, D, G, NW, ST>;
   auto kern = decode_kernel<T, D, G, NW, ST>;
   static bool attr_done[64] = {};
@@ -689,6 +742,7 @@ extern "C" PA_API int pa_decode(void* out, const void* q, const void* k_cache, c
   prm.num_blocks = num_blocks;
   prm.partition = 0;
   prm.num_parts = 1;
+  prm.longest_first = num_seqs > 1 && num_seqs <= PA_DECODE_LPT_MAX_SEQS;
   return run_decode(prm, head_dim, scale, dtype, 1, (cudaStream_t)stream);
 }
 
@@ -729,7 +783,7 @@ namespace pa {
 template <typename T>
 int launch_merge(void* out, const float* po, const float* pm, const float* pl, const int32_t* lens, int rows,
                  int Hq, int D, int partition, int np, cudaStream_t s) {
-  constexpr int MW = 4;
+  constexpr int MW = 8;
   if (D == 64)
     merge_kernel<T, 64, MW><<<rows, MW * 32, 0, s>>>(static_cast<T*>(out), po, pm, pl, lens, Hq, partition, np);
   else if (D == 128)

@@ -67,6 +67,10 @@ template <> struct Mma<__nv_bfloat16> {
     __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
     return *reinterpret_cast<uint32_t*>(&h);
   }
+  // Sum of the two rounded values in a packed pair (exact in fp32).
+  __device__ static inline float sum2(uint32_t u) {
+    return __uint_as_float(u << 16) + __uint_as_float(u & 0xffff0000u);
+  }
 };
 template <> struct Mma<__half> {
   __device__ static inline void run(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
@@ -79,6 +83,10 @@ template <> struct Mma<__half> {
   __device__ static inline uint32_t pack(float x, float y) {
     __half2 h = __floats2half2_rn(x, y);
     return *reinterpret_cast<uint32_t*>(&h);
+  }
+  __device__ static inline float sum2(uint32_t u) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u));
+    return f.x + f.y;
   }
 };
 
@@ -247,10 +255,13 @@ prefill_kernel(const Params p) {
     for (int n = 0; n < NT; ++n) {
       const float p0 = exp2f(s[n][0] - mu0), p1 = exp2f(s[n][1] - mu0);
       const float p2 = exp2f(s[n][2] - mu1), p3 = exp2f(s[n][3] - mu1);
-      rs0 += p0 + p1;
-      rs1 += p2 + p3;
-      pa[n / 2][(n & 1) * 2 + 0] = Mma<T>::pack(p0, p1);
-      pa[n / 2][(n & 1) * 2 + 1] = Mma<T>::pack(p2, p3);
+      // P enters the PV product rounded to the input type; the row sum is
+      // taken over the same rounded values so the weights stay normalised.
+      const uint32_t u01 = Mma<T>::pack(p0, p1), u23 = Mma<T>::pack(p2, p3);
+      pa[n / 2][(n & 1) * 2 + 0] = u01;
+      pa[n / 2][(n & 1) * 2 + 1] = u23;
+      rs0 += Mma<T>::sum2(u01);
+      rs1 += Mma<T>::sum2(u23);
     }
     l0 = l0 * a0 + rs0;
     l1 = l1 * a1 + rs1;

@@ -46,10 +46,11 @@ def assert_close(got: torch.Tensor, ref: np.ndarray, dtype: str, what: str = "")
 
 
 def small_batch(seed, dtype="f16", D=128, G=4, B=16, Hkv=2, lens=(1, 15, 16, 17, 100, 333, 700), chunk=1,
-                poison=float("nan"), q_std=1.0, shared_prefix_tokens=0, shared_group=0):
+                poison=float("nan"), q_std=1.0, shared_prefix_tokens=0, shared_group=0, pool_factor=1.25):
     return W.make_batch(f"small_s{seed}", list(lens), num_q_heads=G * Hkv, num_kv_heads=Hkv, head_dim=D,
                         block_size=B, dtype=dtype, seed=seed, chunk=chunk, poison=poison, q_std=q_std,
-                        shared_prefix_tokens=shared_prefix_tokens, shared_group=shared_group)
+                        shared_prefix_tokens=shared_prefix_tokens, shared_group=shared_group,
+                        pool_factor=pool_factor)
 
 
 def permute_pool(batch, seed=7):

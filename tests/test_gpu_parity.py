@@ -144,7 +144,8 @@ def test_decode_block_permutation_bit_identical():
 
 
 def test_decode_shared_blocks_equal_private_copies():
-    b = small_batch(seed=71, B=16, lens=(300, 200, 129, 50), shared_prefix_tokens=128, shared_group=3)
+    b = small_batch(seed=71, B=16, lens=(300, 200, 129, 50), shared_prefix_tokens=128, shared_group=3,
+                    pool_factor=3.0)
     out1, _, _ = run_gpu(b, partition=None)
     # give sequences 1 and 2 private copies of the 8 shared blocks
     b2 = b.to("cpu")
