@@ -5,7 +5,7 @@ given (device, dtype, contiguity), derives the sizes the C ABI wants from
 their shapes, and calls the entry point of the same name in libpa.so on the
 current CUDA stream. All arithmetic runs in the library's CUDA kernels; there
 is no CPU fallback. Importing the package fails loudly if libpa.so is missing
-(build it with `python -m paged_kv_cache_475_b200.build`).
+(build it with `python paged_kv_cache_475_b200/build.py`).
 
 The C declarations and their contracts are in include/pa.h.
 """
@@ -21,7 +21,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("PA_LIBRARY") or os.path.join(_PKG, "libpa.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_475_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python paged_kv_cache_475_b200/build.py`")
 _lib = ctypes.CDLL(LIB_PATH)
 
 PA_F32, PA_F16, PA_BF16 = 0, 1, 2
@@ -51,7 +51,7 @@ _SIGS = {
 for _name, _args in _SIGS.items():
     _fn = getattr(_lib, _name)
     _fn.argtypes = _args
-    _fn.restype = ctypes.c_char_p if _name == "pa_status_string" else _i
+    _fn.restype = {"pa_status_string": ctypes.c_char_p, "pa_noalloc_scratch_bytes": _sz}.get(_name, _i)
 
 
 class PagedAttentionError(RuntimeError):

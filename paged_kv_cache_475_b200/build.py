@@ -1,6 +1,7 @@
 """Build libpa.so in-tree with nvcc for sm_100a (B200).
 
-python -m paged_kv_cache_475_b200.build [--force] [--verbose]
+python paged_kv_cache_475_b200/build.py [--force] [--verbose]
+(run it as a script: importing the package loads libpa.so, which may not exist yet)
 
 Sources are compiled in parallel into _build/ (git-ignored) and linked into
 paged_kv_cache_475_b200/libpa.so. A rebuild happens only when a source or the
@@ -51,7 +52,7 @@ def build(force: bool = False, verbose: bool = False, defines=(), lib: str = LIB
 
     defines: extra -D macros (tuning variants), written to `lib` with objects in `objdir`.
     """
-    if not force and lib == LIB and not _stale():
+    if not force and os.path.abspath(lib) == LIB and not _stale():
         return LIB
     os.makedirs(objdir, exist_ok=True)
     cc = nvcc()

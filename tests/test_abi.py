@@ -6,9 +6,19 @@ import re
 
 import pytest
 
-from paged_kv_cache_475_b200 import build as B
-
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _build_module():
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location("pa_build", os.path.join(ROOT, "paged_kv_cache_475_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+B = _build_module()
 
 
 @pytest.fixture(scope="module")
