@@ -197,6 +197,39 @@ PA_API int pa_prefill_chunk(void* out, const void* q, const void* k_cache, const
                             int num_blocks, float scale, pa_dtype dtype, void* stream);
 
 /*
+ * pa_decode_splitkv_noalloc - split-KV decode and merge in one call, with no
+ * device memory allocated by the caller or by the library. (The pages have
+ * no counterpart of this entry point; it exists for callers that cannot
+ * allocate.)
+ *
+ * Same result as pa_decode_splitkv followed by pa_merge, written to `out`
+ * [N, Hq, D]. It is meant for callers that cannot provide a workspace: a
+ * plugin or FFI host with no device allocator at hand, a serving runtime
+ * that has already handed all free HBM to its KV block pool, or a
+ * latency-critical loop that cannot afford cudaMalloc's implicit device
+ * synchronisation. The partials live instead in a fixed array inside the
+ * library's own device memory, pa_noalloc_scratch_bytes() = 16 MiB on every
+ * GPU that loads the library, held until the process exits. The call needs
+ * N * Hq * num_partitions * (D + 2) * 4 bytes of it (each part rounded up to
+ * 256 bytes); larger requests return PA_ERR_WORKSPACE and launch nothing.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture begins. Every call on a device shares the one array: calls whose
+ * kernels overlap on the GPU (other streams, other host threads) race and
+ * must be serialised by the caller. Nothing in the array needs clearing: each
+ * call writes every partial it later reads.
+ */
+PA_API int pa_decode_splitkv_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_tables, int max_blocks_per_seq,
+                                     const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                     int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                     int partition_size, int num_partitions, float scale,
+                                     pa_dtype dtype, void* stream);
+
+/* Size in bytes of the per-device array pa_decode_splitkv_noalloc works in. */
+PA_API size_t pa_noalloc_scratch_bytes(void);
+
+/*
  * pa_read_error_flags - read (and optionally clear) the device error word of
  * the current device. Synchronises the device. Returns PA_OK or PA_ERR_CUDA.
  */

@@ -44,6 +44,9 @@ _SIGS = {
                           _i, _vp],
     "pa_merge": [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp],
     "pa_prefill_chunk": [_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp],
+    "pa_decode_splitkv_noalloc": [_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
+                                  _vp],
+    "pa_noalloc_scratch_bytes": [],
     "pa_read_error_flags": [ctypes.POINTER(ctypes.c_uint32), _i],
     "pa_status_string": [_i],
     "pa_version": [],
@@ -196,6 +199,25 @@ def pa_prefill_chunk(out, q, k_cache, v_cache, block_tables, context_lens, scale
     _check(_lib.pa_prefill_chunk(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                                  block_tables.shape[1], _ptr(context_lens), N, q.shape[1], q.shape[2], Hkv, D, B,
                                  P, float(scale), _dtype_code(q), _stream(stream)), "pa_prefill_chunk")
+
+
+def pa_decode_splitkv_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, partition_size: int,
+                              num_partitions: int, scale: float, stream=None):
+    """Split-KV decode + merge into out [N, Hq, D] with the partials in the library's fixed
+    per-device array (no workspace from the caller); see include/pa.h for its limits."""
+    _need(q, "q", None, 3)
+    _need(out, "out", q.dtype, 3)
+    P, Hkv, B, D, N = _cache_dims(q, k_cache, v_cache, block_tables, context_lens)
+    if q.shape[0] != N or q.shape[2] != D or out.shape != q.shape:
+        raise ValueError("q/out must be [N, Hq, D]")
+    _check(_lib.pa_decode_splitkv_noalloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                          block_tables.shape[1], _ptr(context_lens), N, q.shape[1], Hkv, D, B, P,
+                                          int(partition_size), int(num_partitions), float(scale), _dtype_code(q),
+                                          _stream(stream)), "pa_decode_splitkv_noalloc")
+
+
+def pa_noalloc_scratch_bytes() -> int:
+    return _lib.pa_noalloc_scratch_bytes()
 
 
 def pa_read_error_flags(clear: bool = True) -> int:

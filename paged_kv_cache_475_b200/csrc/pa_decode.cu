@@ -24,6 +24,8 @@
 //    probabilities through a 16 x G shared-memory slot, then P.V with each
 //    lane owning D/32 output dims for all G heads;
 //  * the warps' (m, l, o) states merge in shared memory at the end.
+#include <mutex>
+
 #include "pa_common.cuh"
 
 namespace pa {
@@ -815,4 +817,83 @@ extern "C" PA_API int pa_merge(void* out, const float* part_o, const float* part
                                                      num_q_heads, head_dim, partition_size, num_partitions, s);
   }
   return PA_ERR_DTYPE;
+}
+
+// ---------------------------------------------------------------------------
+// pa_decode_splitkv_noalloc: split-KV decode plus merge without any device
+// allocation by the caller or by the library.
+//
+// Some callers cannot hand this library a workspace: a plugin or FFI host
+// that exposes no device allocator, a serving runtime that has already given
+// all free HBM to its KV block pool, or a latency-critical loop where
+// cudaMalloc's implicit device synchronisation is not acceptable. For them
+// the partials of the split-KV pass live in a fixed array in the library's
+// own device memory (kNoAllocScratchBytes per GPU that loads the library,
+// held until the process exits). The caller still passes q, the caches, the
+// tables and the output.
+// ---------------------------------------------------------------------------
+namespace pa {
+namespace noalloc {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+static unsigned char* g_scratch_dev[kMaxDevices] = {};
+static std::mutex g_scratch_mu;
+
+// Device address of g_scratch on the current device. In host code the name
+// g_scratch is only a host-side stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+static int scratch_address(unsigned char** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_dev[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return PA_ERR_CUDA;
+    g_scratch_dev[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = g_scratch_dev[dev];
+  return PA_OK;
+}
+
+}  // namespace noalloc
+}  // namespace pa
+
+extern "C" PA_API size_t pa_noalloc_scratch_bytes(void) { return pa::noalloc::kNoAllocScratchBytes; }
+
+extern "C" PA_API int pa_decode_splitkv_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                                const int32_t* block_tables, int max_blocks_per_seq,
+                                                const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                                int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                                int partition_size, int num_partitions, float scale,
+                                                pa_dtype dtype, void* stream) {
+  int st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                             num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, dtype);
+  if (st != PA_OK || num_seqs == 0) return st;
+  if (!out) return PA_ERR_NULL;
+  if (partition_size <= 0 || partition_size % kTile || num_partitions <= 0) return PA_ERR_WORKSPACE;
+  if (num_seqs > 65535) return PA_ERR_SHAPE;
+  // Partials: o [rows, NP, D], then m and l [rows, NP], each start 256-byte aligned.
+  const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads;
+  const size_t cells = rows * static_cast<size_t>(num_partitions);
+  const size_t o_bytes = (cells * head_dim * sizeof(float) + 255) & ~size_t(255);
+  const size_t ml_bytes = (cells * sizeof(float) + 255) & ~size_t(255);
+  if (o_bytes + 2 * ml_bytes > pa::noalloc::kNoAllocScratchBytes) return PA_ERR_WORKSPACE;
+  unsigned char* base = nullptr;
+  st = pa::noalloc::scratch_address(&base);
+  if (st != PA_OK) return st;
+  float* part_o = reinterpret_cast<float*>(base);
+  float* part_m = reinterpret_cast<float*>(base + o_bytes);
+  float* part_l = reinterpret_cast<float*>(base + o_bytes + ml_bytes);
+  // Every partition p < num_partitions of every row is written by the split
+  // pass (empty ones as m = -inf, l = 0, o = 0) before the merge reads it, so
+  // nothing left in the array by an earlier call is ever read.
+  st = pa_decode_splitkv(part_o, part_m, part_l, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                         context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                         partition_size, num_partitions, scale, dtype, stream);
+  if (st != PA_OK) return st;
+  return pa_merge(out, part_o, part_m, part_l, context_lens, num_seqs, num_q_heads, head_dim, partition_size,
+                  num_partitions, dtype, stream);
 }
