@@ -109,7 +109,7 @@ def measured_peaks():
 
 def kernel_traffic(kernel_key):
     """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
         return None
     with open(p) as f:
@@ -198,26 +198,26 @@ def dist_init(args):
     return world, rank, local
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
     import torch
 
     if world == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def sum_over_ranks(x, world):
+def sum_over_ranks(x, world, device="cuda"):
     import torch
 
     if world == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
 
