@@ -125,22 +125,28 @@ __device__ inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
-// Bounded wait on a phase of an mbarrier. Returns false if the phase did not
-// complete within `limit` polls (the caller records PA_DEVERR_WAIT).
-__device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = (1u << 24)) {
+// Bounded wait on a phase of an mbarrier: gives up after about `max_cycles`
+// SM clock cycles (~2 s at 1.9 GHz by default), however long each try_wait
+// suspends. Returns false on timeout (the caller records PA_DEVERR_WAIT).
+__device__ inline bool mbar_try(uint32_t a, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(a), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+__device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity, long long max_cycles = 4000000000LL) {
   const uint32_t a = smem_addr(bar);
-  for (uint32_t i = 0; i < limit; ++i) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (done) return true;
+  if (mbar_try(a, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try(a, parity)) return true;
+    if (clock64() - t0 > max_cycles) return false;
   }
-  return false;
 }
 
 // Global -> shared bulk copy completing on an mbarrier (byte count, 16-byte

@@ -357,7 +357,7 @@ decode_kernel(const DecodeParams p) {
   int k = 0;
   for (; k < my_tiles; ++k) {
     const int s = k % STAGES;
-    if (!mbar_wait(&bars[s], (k / STAGES) & 1)) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[s], (k / STAGES) & 1))) {
       if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
       aborted = true;
       break;
@@ -492,7 +492,7 @@ decode_kernel(const DecodeParams p) {
   if (aborted) {
     // Let this warp's copies still in flight land before the CTA exits.
     const int issued = my_tiles < k + STAGES ? my_tiles : k + STAGES;
-    for (int kk = k; kk < issued; ++kk) mbar_wait(&bars[kk % STAGES], (kk / STAGES) & 1, 1u << 20);
+    for (int kk = k; kk < issued; ++kk) mbar_wait(&bars[kk % STAGES], (kk / STAGES) & 1, 400000000LL);
   }
 
   // ---- per-warp finish: l for every head -------------------------------------

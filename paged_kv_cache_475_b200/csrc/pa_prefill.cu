@@ -1,85 +1,187 @@
-// Chunked prefill over a paged context: pa_prefill_chunk (tensor cores).
+// Chunked prefill over a paged context on the 5th-generation tensor cores
+// (tcgen05 + TMEM + TMA), sm_100a.
 //
-// Query i of a C-token chunk sits at position L - C + i and attends to keys
-// 0..L-C+i: the whole earlier context and the chunk's own keys up to itself.
-// This is eq. (4) of "Flash Attention vs Paged Attention" (算法原理: the block
-// sum stops at the block holding the query, cut at its own token), evaluated
-// with the online softmax and fused QK^T / softmax / PV of "FlashAttention y
-// PagedAttention" (FlashAttention "Cómo funciona"); key tiles wholly past a
-// query tile are never computed and the causal mask is applied in registers
-// (kernel fusion section of the same Chinese page).
+// What it computes (pa_prefill_chunk in include/pa.h): query
+// i of a C-token chunk sits at position L - C + i and attends to keys
+// 0..L-C+i; eq. (4) of "Flash Attention vs Paged Attention" (算法原理) with the
+// online softmax and fused QK^T / softmax / PV of "FlashAttention y
+// PagedAttention" (FlashAttention "Cómo funciona"); key tiles past a query
+// tile are never computed, the causal mask is applied in registers.
 //
-// Design: one CTA (4 warps) per (sequence, KV head, query tile). The 64 rows
-// of a query tile are (query, head) pairs of one GQA group, so every K/V tile
-// gathered from the pool serves all G heads. K/V tiles of 64 tokens are
-// gathered page by page with 16-byte cp.async (zero-filled past the context),
-// stored XOR-swizzled for conflict-free ldmatrix, double-buffered, and fed to
-// bf16/f16 mma.sync m16n8k16 with fp32 accumulation.
+// One CTA (6 warps) per (sequence, KV head, 128-row query tile); the 128 rows
+// are (query, head) pairs of one GQA group, so each gathered K/V page serves
+// all G heads of the group. Warp roles:
+//   warps 0-3  softmax: thread r owns row r (TMEM lane r); reads its S row
+//              from TMEM, keeps the running max / sum, writes P (bf16/f16) to
+//              shared memory, rescales its O row in TMEM when its max grows by
+//              more than 2^8, and finally writes O / l;
+//   warp 4     producer: TMA tensor copies of the Q tile (once) and of each
+//              128-key K/V tile, gathered page by page through the block table
+//              (one 2-D box of min(B,16) rows per page chunk, 128-byte swizzle;
+//              chunks past the context read out of range and land as zeros);
+//   warp 5     MMA: one thread issues S = Q K^T into a double-buffered TMEM
+//              accumulator and O += P V into a TMEM accumulator (M = 128,
+//              N = 128, K = 16 per instruction), completions via tcgen05.commit
+//              on mbarriers; it zeroes V rows past the context in the last
+//              partial page chunk before they reach the PV product.
+// Every mbarrier wait is bounded; a timeout sets PA_DEVERR_WAIT and the CTA
+// drains, frees its TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "pa_common.cuh"
 
 namespace pa {
-namespace prefill {
+namespace tc {
 
-constexpr int kBM = 64;   // query rows per CTA
-constexpr int kBN = 64;   // keys per tile
-constexpr int kWarps = 4;
+constexpr int kM = 128;        // query rows per CTA = TMEM lanes
+constexpr int kN = 128;        // keys per tile
+constexpr int kStages = 2;     // K and V rings
+constexpr int kThreads = 192;  // 4 softmax warps + producer + MMA
+constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleLog2 = 8.0f;  // keep a stale max until the true one is 2^8 larger
 
 struct Params {
   void* out;
-  const void* q;
-  const void* k_cache;
-  const void* v_cache;
   const int32_t* block_tables;
   const int32_t* context_lens;
   unsigned int* err;
   int max_blocks, num_seqs, chunk, num_q_heads, num_kv_heads, block_size, num_blocks;
+  int chunk_rows;      // rows per TMA box = min(B, 16)
+  int oob_row;         // a row coordinate past the pool: TMA reads zeros there
   float scale_log2;
 };
 
-__device__ inline void cp_async16(uint32_t dst, const void* src, bool fill) {
-  const int n = fill ? 16 : 0;  // src-size 0: the 16 bytes are zero-filled
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
-}
-__device__ inline void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ inline void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+template <int D>
+struct Smem {
+  static constexpr int kQ = kM * D * 2;   // D/64 atoms of [128 rows x 128 B]
+  static constexpr int kKV = kN * D * 2;  // one K or V tile
+  static constexpr int kP = kM * kN * 2;  // two atoms of [128 rows x 128 B]
+  static constexpr int oQ = 0;
+  static constexpr int oK = oQ + kQ;
+  static constexpr int oV = oK + kStages * kKV;
+  static constexpr int oP = oV + kStages * kKV;
+  static constexpr int oBar = oP + kP;
+  // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full, o_done
+  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2;
+  static constexpr int oTmem = oBar + kNumBars * 8;
+  static constexpr int kUsed = oTmem + 16;
+  static constexpr int kAlloc = kUsed + 1024;  // room to align the base to 1024 B
+};
 
-__device__ inline void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+// ---------------------------------------------------------------------------
+// tcgen05 / TMA wrappers (inline PTX)
+// ---------------------------------------------------------------------------
+__device__ inline void tmem_alloc(uint32_t* slot, int cols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)), "r"(cols)
+               : "memory");
 }
-__device__ inline void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+__device__ inline void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ inline void tmem_dealloc(uint32_t taddr, int cols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+__device__ inline void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ inline void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ inline void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ inline void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
 }
 
-template <typename T> struct Mma;
-template <> struct Mma<__nv_bfloat16> {
-  __device__ static inline void run(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-  }
+__device__ inline void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16, one CTA.
+__device__ inline void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc), "r"(0), "r"(0), "r"(0), "r"(0)
+      : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ inline void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ inline void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+      ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+__device__ inline void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ inline void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ inline void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ inline void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), version 1.
+// lbo/sbo in 16-byte units.
+__device__ inline uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(lbo & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>(sbo & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulate, A/B both `fmt`
+// (0 = f16, 1 = bf16), A K-major, B K-major (b_mn = 0) or MN-major (1).
+__host__ __device__ constexpr uint32_t idesc_f16(uint32_t fmt, uint32_t b_mn, int M, int N) {
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | (b_mn << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+template <typename T> struct Fmt;
+template <> struct Fmt<__nv_bfloat16> {
+  static constexpr uint32_t kCode = 1;
   __device__ static inline uint32_t pack(float x, float y) {
     __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
     return *reinterpret_cast<uint32_t*>(&h);
   }
-  // Sum of the two rounded values in a packed pair (exact in fp32).
   __device__ static inline float sum2(uint32_t u) {
     return __uint_as_float(u << 16) + __uint_as_float(u & 0xffff0000u);
   }
 };
-template <> struct Mma<__half> {
-  __device__ static inline void run(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-  }
+template <> struct Fmt<__half> {
+  static constexpr uint32_t kCode = 0;
   __device__ static inline uint32_t pack(float x, float y) {
     __half2 h = __floats2half2_rn(x, y);
     return *reinterpret_cast<uint32_t*>(&h);
@@ -90,265 +192,438 @@ template <> struct Mma<__half> {
   }
 };
 
-// Byte offset of 16-byte chunk c of row r in a swizzled [rows][D] tile.
-template <int D>
-__device__ inline uint32_t swz(int r, int c) {
-  constexpr int RC = D * 2 / 16;  // chunks per row
-  return static_cast<uint32_t>(r * RC * 16 + ((c ^ (r & 7)) * 16));
+// Every wait of this kernel gives up after about 2 s and is made warp-uniform,
+// so a timeout can never split a warp at a __syncwarp.
+__device__ inline bool wait_all(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kWarps * 32)
-prefill_kernel(const Params p) {
-  constexpr int RC = D * 2 / 16;           // 16-byte chunks per row
-  constexpr int QT = kBM / G;              // queries per CTA
-  constexpr int KS = D / 16;               // k-steps over the head dim
-  constexpr int NT = kBN / 8;              // score n-tiles per key tile
-  constexpr int DT = D / 8;                // output n-tiles
-  constexpr int kTileBytes = kBN * D * 2;
-  extern __shared__ __align__(128) unsigned char smem[];
-  unsigned char* sQ = smem;
-  unsigned char* sK = smem + kBM * D * 2;           // [2][kBN][D]
-  unsigned char* sV = sK + 2 * kTileBytes;          // [2][kBN][D]
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  using S = Smem<D>;
+  constexpr int QT = kM / G;       // queries per CTA
+  constexpr int KA = D / 64;       // 128-byte atoms along the head dim
+  constexpr int KS = D / 16;       // MMA k-steps of S = Q K^T
+  constexpr uint32_t kIdescS = idesc_f16(Fmt<T>::kCode, 0, kM, kN);
+  constexpr uint32_t kIdescO = idesc_f16(Fmt<T>::kCode, 1, kM, D);
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int num_qt = gridDim.x;
-  const int qt = num_qt - 1 - blockIdx.x;   // heaviest (latest) query tiles first
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  unsigned char* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  const uint32_t sb = smem_addr(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::oBar);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + kStages;
+  uint64_t* v_full = k_empty + kStages;
+  uint64_t* v_empty = v_full + kStages;
+  uint64_t* s_full = v_empty + kStages;   // [2]
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = p_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::oTmem);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = gridDim.x - 1 - blockIdx.x;  // latest (heaviest) query tiles first
   const int kvh = blockIdx.y, b = blockIdx.z;
   const int C = p.chunk, B = p.block_size;
-
   int L = p.context_lens[b];
   if (L < 0 || L > p.max_blocks * B) {
-    if (tid == 0) set_error(p.err, PA_DEVERR_CONTEXT);
+    if (threadIdx.x == 0) set_error(p.err, PA_DEVERR_CONTEXT);
     L = L < 0 ? 0 : p.max_blocks * B;
   }
-  const int i0 = qt * QT;                   // first query of the tile
-  const int q_hi = min(C, i0 + QT);         // one past the last query
-  const int pos_lo = L - C + i0;            // position of the first query
-  const int pos_hi = L - C + q_hi - 1;      // position of the last query
+  const int i0 = qt * QT;
+  const int q_hi = min(C, i0 + QT);
+  const int pos_lo = L - C + i0;
+  const int pos_hi = L - C + q_hi - 1;
   const int n_keys = pos_hi + 1 > 0 ? pos_hi + 1 : 0;
-  const int n_ktiles = (n_keys + kBN - 1) / kBN;
+  const int n_tiles = (n_keys + kN - 1) / kN;
 
-  const T* qg = static_cast<const T*>(p.q);
-  const T* kc = static_cast<const T*>(p.k_cache);
-  const T* vc = static_cast<const T*>(p.v_cache);
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(p_full, 4);
+    mbar_init(o_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS0 = tmem, tS1 = tmem + kN, tO = tmem + 2 * kN;
+
+  const uint32_t sQ = sb + S::oQ, sK = sb + S::oK, sV = sb + S::oV, sP = sb + S::oP;
   const int32_t* bt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
 
-  // ---- Q tile: row r = (query i0 + r/G, head kvh*G + r%G) -------------------
-  for (int idx = tid; idx < kBM * RC; idx += kWarps * 32) {
-    const int r = idx / RC, c = idx % RC;
-    const int i = i0 + r / G;
-    const bool ok = i < C;
-    const T* src = qg + ((static_cast<int64_t>(b) * C + (ok ? i : 0)) * p.num_q_heads + kvh * G + r % G) * D + c * 8;
-    cp_async16(smem_addr(sQ) + swz<D>(r, c), src, ok);
-  }
-  cp_async_commit();
-
-  auto load_kv = [&](int kt, int buf) {
-    const int t0 = kt * kBN;
-    const uint32_t kbase = smem_addr(sK + buf * kTileBytes);
-    const uint32_t vbase = smem_addr(sV + buf * kTileBytes);
-    for (int idx = tid; idx < kBN * RC; idx += kWarps * 32) {
-      const int r = idx / RC, c = idx % RC;
-      const int t = t0 + r;
-      bool ok = t < L;
-      int64_t off = 0;
-      if (ok) {
-        const int id = bt[t / B];
-        if (id < 0 || id >= p.num_blocks) {
-          set_error(p.err, PA_DEVERR_BLOCK_ID);
-          ok = false;
+  if (warp == 4) {
+    // ------------------------------ producer ------------------------------
+    if (n_tiles > 0) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(q_full, S::kQ);
+        for (int a = 0; a < KA; ++a)
+          tma_load_3d(sQ + a * (kM * 128), &tm_q, a * 64, kvh * G, b * C + i0, q_full);
+      }
+      const int R = p.chunk_rows;
+      const int chunks = kN / R;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int st = j % kStages;
+        const uint32_t par = ((j / kStages) & 1) ^ 1;
+        bool ok = wait_all(&k_empty[st], par);
+        if (lane == 0) mbar_arrive_expect_tx(&k_full[st], S::kKV);
+        __syncwarp();
+        // lane c gathers page chunk c (and c + 32 when B = 8) of this tile
+        int ys[2] = {p.oob_row, p.oob_row};
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int c = lane + 32 * u;
+          if (c < chunks) {
+            const int t0 = j * kN + c * R;
+            if (t0 < L) {
+              const int id = bt[t0 / B];
+              if (id >= 0 && id < p.num_blocks)
+                ys[u] = (id * p.num_kv_heads + kvh) * B + (t0 % B);
+              else
+                set_error(p.err, PA_DEVERR_BLOCK_ID);
+            }
+            for (int a = 0; a < KA; ++a)
+              tma_load_2d(sK + st * S::kKV + a * (kN * 128) + c * R * 128, &tm_k, a * 64, ys[u], &k_full[st]);
+          }
+        }
+        ok = wait_all(&v_empty[st], par) && ok;
+        if (lane == 0) mbar_arrive_expect_tx(&v_full[st], S::kKV);
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int c = lane + 32 * u;
+          if (c < chunks)
+            for (int a = 0; a < KA; ++a)
+              tma_load_2d(sV + st * S::kKV + a * (kN * 128) + c * R * 128, &tm_v, a * 64, ys[u], &v_full[st]);
+        }
+        if (!ok) {
+          if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
+          break;
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // -------------------------------- MMA ---------------------------------
+    bool ok = n_tiles == 0 || wait_all(q_full, 0);
+    auto issue_pv = [&](int k) -> bool {
+      const int st = k % kStages;
+      bool good = wait_all(p_full, k & 1);
+      good = wait_all(&v_full[st], (k / kStages) & 1) && good;
+      if (!good) return false;
+      // V rows past the context inside the last page chunk hold whatever the
+      // pool holds there; P is 0 for them but 0 * NaN is NaN, so zero them.
+      const int R = p.chunk_rows;
+      const int z0 = L - k * kN;
+      if (z0 > 0 && z0 < kN && (L % R) != 0) {
+        const int z1 = min(kN, ((L + R - 1) / R) * R - k * kN);
+        const int n16 = (z1 - z0) * KA * 8;  // 16-byte pieces
+        for (int e = lane; e < n16; e += 32) {
+          const int row = z0 + e / (KA * 8), rest = e % (KA * 8);
+          const int a = rest / 8, c = rest % 8;
+          uint4* dst = reinterpret_cast<uint4*>(smem + S::oV + st * S::kKV + a * (kN * 128) + row * 128 + c * 16);
+          *dst = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      tc_fence_after();
+      if (lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < kN / 16; ++kk) {
+          const uint64_t ad = sw128_desc(sP + (kk / 4) * (kM * 128) + (kk % 4) * 32, 1, 64);
+          const uint64_t bd = sw128_desc(sV + st * S::kKV + kk * 2048, (kN * 128) >> 4, 64);
+          tc_mma(tO, ad, bd, kIdescO, (k > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(o_done);
+        tc_commit(&v_empty[st]);
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int j = 0; j < n_tiles && ok; ++j) {
+      const int st = j % kStages;
+      ok = wait_all(&k_full[st], (j / kStages) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t tS = (j & 1) ? tS1 : tS0;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const uint32_t koff = (ks / 4) * (kM * 128) + (ks % 4) * 32;
+          const uint32_t kkoff = (ks / 4) * (kN * 128) + (ks % 4) * 32;
+          const uint64_t ad = sw128_desc(sQ + koff, 1, 64);
+          const uint64_t bd = sw128_desc(sK + st * S::kKV + kkoff, 1, 64);
+          tc_mma(tS, ad, bd, kIdescS, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full[j & 1]);
+        tc_commit(&k_empty[st]);
+      }
+      __syncwarp();
+      if (j > 0) ok = issue_pv(j - 1);
+    }
+    if (ok && n_tiles > 0) ok = issue_pv(n_tiles - 1);
+    if (!ok && lane == 0) set_error(p.err, PA_DEVERR_WAIT);
+  } else {
+    // ------------------------------ softmax -------------------------------
+    const int r = threadIdx.x;                 // row = TMEM lane
+    const int i = i0 + r / G, g = r % G;
+    const int pos = L - C + i;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles && ok; ++j) {
+      ok = wait_all(&s_full[j & 1], (j >> 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tS = ((j & 1) ? tS1 : tS0) + lane_off;
+      const int t0 = j * kN;
+      const bool masked_tile = t0 + kN - 1 > pos_lo;
+      // pass 1: row max of the (masked) raw scores
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kN / 32; ++c) {
+        float v[32];
+        tmem_ld32(tS + c * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const bool cut = masked_tile && (t0 + c * 32 + e > pos);
+          mx = fmaxf(mx, cut ? -INFINITY : v[e]);
+        }
+      }
+      const float m_tile = mx * p.scale_log2;
+      const float m_new = fmaxf(m, m_tile);
+      // Rescale only when the max grows by more than 2^8 (or on the first
+      // finite max); otherwise keep the stale max, which bounds p by 2^8.
+      const bool rescale = (m == -INFINITY) || (m_new > m + kRescaleLog2);
+      const float m_use = rescale ? m_new : m;
+      const float m_sub = m_use == -INFINITY ? 0.f : m_use;
+      const float alpha = exp2f(m - m_sub);  // 0 while nothing was seen yet
+      // pass 2: probabilities, packed to the input type
+      uint32_t pk[kN / 2];
+      float psum = 0.f;
+#pragma unroll
+      for (int c = 0; c < kN / 32; ++c) {
+        float v[32];
+        tmem_ld32(tS + c * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int t = t0 + c * 32 + e;
+          const float a0 = (masked_tile && t > pos) ? -INFINITY : v[e];
+          const float a1 = (masked_tile && t + 1 > pos) ? -INFINITY : v[e + 1];
+          const uint32_t u = Fmt<T>::pack(exp2f(fmaf(a0, p.scale_log2, -m_sub)), exp2f(fmaf(a1, p.scale_log2, -m_sub)));
+          pk[(c * 32 + e) / 2] = u;
+          psum += Fmt<T>::sum2(u);
+        }
+      }
+      l = l * alpha + psum;
+      m = m_use;
+      if (j > 0) {  // PV(j-1) must be done before O is touched or P is overwritten
+        ok = wait_all(o_done, (j - 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        // tcgen05.ld/st are warp-collective: the whole warp takes this branch
+        // when any of its rows needs a rescale (the others multiply by 1).
+        const bool need = rescale && alpha != 1.f;
+        if (__any_sync(0xffffffffu, need)) {
+          const float f = need ? alpha : 1.f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tmem_ld32(tO + lane_off + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= f;
+            tmem_st32(tO + lane_off + c * 32, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      // P row -> shared memory, 128-byte swizzled K-major (2 atoms of 64 keys)
+#pragma unroll
+      for (int c = 0; c < kN / 8; ++c) {
+        const int a = c / 8, cc = c % 8;
+        const uint32_t off = a * (kM * 128) + (r / 8) * 1024 + (r % 8) * 128 + ((cc ^ (r % 8)) * 16);
+        *reinterpret_cast<uint4*>(smem + S::oP + off) =
+            make_uint4(pk[c * 4 + 0], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    // epilogue: out = O / l
+    if (ok && n_tiles > 0) {
+      ok = wait_all(o_done, (n_tiles - 1) & 1);
+      tc_fence_after();
+    }
+    if (!ok) {
+      set_error(p.err, PA_DEVERR_WAIT);
+    } else {
+      // Every thread of the warp reads its O row (warp-collective tcgen05.ld);
+      // only rows of real queries (i < C) are stored.
+      const bool store = i < C;
+      const float inv = (l > 0.f && n_tiles > 0) ? 1.f / l : 0.f;
+      T* orow = static_cast<T*>(p.out) +
+                ((static_cast<int64_t>(b) * C + (store ? i : 0)) * p.num_q_heads + kvh * G + g) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        if (n_tiles > 0) {
+          tmem_ld32(tO + lane_off + c * 32, o);
+          tmem_wait_ld();
         } else {
-          off = ((static_cast<int64_t>(id) * p.num_kv_heads + kvh) * B + t % B) * D + c * 8;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0.f;
+        }
+        if (!store) continue;
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          uint4 v = make_uint4(Fmt<T>::pack(o[e] * inv, o[e + 1] * inv), Fmt<T>::pack(o[e + 2] * inv, o[e + 3] * inv),
+                               Fmt<T>::pack(o[e + 4] * inv, o[e + 5] * inv), Fmt<T>::pack(o[e + 6] * inv, o[e + 7] * inv));
+          *reinterpret_cast<uint4*>(orow + c * 32 + e) = v;
         }
       }
-      cp_async16(kbase + swz<D>(r, c), kc + off, ok);
-      cp_async16(vbase + swz<D>(r, c), vc + off, ok);
     }
-  };
+  }
 
-  if (n_ktiles > 0) load_kv(0, 0);
-  cp_async_commit();
-
-  // ---- per-thread row state ---------------------------------------------------
-  const int r0 = warp * 16 + (lane >> 2);   // this thread's rows: r0 and r0 + 8
-  const int pos_r0 = L - C + i0 + r0 / G;
-  const int pos_r1 = L - C + i0 + (r0 + 8) / G;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  float o[DT][4];
-#pragma unroll
-  for (int n = 0; n < DT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-
-  uint32_t qa[KS][4];
-  cp_async_wait<1>();
+  tc_fence_before();
   __syncthreads();
-#pragma unroll
-  for (int ks = 0; ks < KS; ++ks) {
-    const int r = warp * 16 + (lane & 15);
-    const int c = ks * 2 + (lane >> 4);
-    ldsm_x4(smem_addr(sQ) + swz<D>(r, c), qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
-  }
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+}
 
-  for (int kt = 0; kt < n_ktiles; ++kt) {
-    const int buf = kt & 1;
-    if (kt + 1 < n_ktiles) load_kv(kt + 1, buf ^ 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
+// ---------------------------------------------------------------------------
+// Host side: tensor maps and launch
+// ---------------------------------------------------------------------------
 
-    const uint32_t kb = smem_addr(sK + buf * kTileBytes);
-    const uint32_t vb = smem_addr(sV + buf * kTileBytes);
-    const int t0 = kt * kBN;
-
-    // -- S = Q K^T (16 x 64 per warp) --
-    float s[NT][4];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-#pragma unroll
-      for (int np = 0; np < NT / 2; ++np) {
-        uint32_t b0, b1, b2, b3;
-        const int r = np * 16 + (lane & 7) + ((lane >> 4) << 3);
-        const int c = ks * 2 + ((lane >> 3) & 1);
-        ldsm_x4(kb + swz<D>(r, c), b0, b1, b2, b3);
-        Mma<T>::run(s[2 * np], qa[ks], b0, b1);
-        Mma<T>::run(s[2 * np + 1], qa[ks], b2, b3);
-      }
-    }
-
-    // -- causal mask (only tiles reaching past the first query's position) --
-    const bool need_mask = t0 + kBN - 1 > pos_lo;
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float v = s[n][e] * p.scale_log2;
-        if (need_mask) {
-          const int t = t0 + n * 8 + (lane & 3) * 2 + (e & 1);
-          const int pr = e < 2 ? pos_r0 : pos_r1;
-          if (t > pr) v = -INFINITY;
-        }
-        s[n][e] = v;
-      }
-    }
-
-    // -- online softmax --
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      mx0 = fmaxf(mx0, fmaxf(s[n][0], s[n][1]));
-      mx1 = fmaxf(mx1, fmaxf(s[n][2], s[n][3]));
-    }
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
-    const float a0 = exp2f(m0 - mu0), a1 = exp2f(m1 - mu1);
-    m0 = mn0;
-    m1 = mn1;
-    float rs0 = 0.f, rs1 = 0.f;
-    uint32_t pa[NT / 2][4];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      const float p0 = exp2f(s[n][0] - mu0), p1 = exp2f(s[n][1] - mu0);
-      const float p2 = exp2f(s[n][2] - mu1), p3 = exp2f(s[n][3] - mu1);
-      // P enters the PV product rounded to the input type; the row sum is
-      // taken over the same rounded values so the weights stay normalised.
-      const uint32_t u01 = Mma<T>::pack(p0, p1), u23 = Mma<T>::pack(p2, p3);
-      pa[n / 2][(n & 1) * 2 + 0] = u01;
-      pa[n / 2][(n & 1) * 2 + 1] = u23;
-      rs0 += Mma<T>::sum2(u01);
-      rs1 += Mma<T>::sum2(u23);
-    }
-    l0 = l0 * a0 + rs0;
-    l1 = l1 * a1 + rs1;
-#pragma unroll
-    for (int n = 0; n < DT; ++n) {
-      o[n][0] *= a0; o[n][1] *= a0;
-      o[n][2] *= a1; o[n][3] *= a1;
-    }
-
-    // -- O += P V --
-#pragma unroll
-    for (int kk = 0; kk < kBN / 16; ++kk) {
-#pragma unroll
-      for (int dp = 0; dp < DT / 2; ++dp) {
-        uint32_t b0, b1, b2, b3;
-        const int r = kk * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-        const int c = dp * 2 + (lane >> 4);
-        ldsm_x4_t(vb + swz<D>(r, c), b0, b1, b2, b3);
-        Mma<T>::run(o[2 * dp], pa[kk], b0, b1);
-        Mma<T>::run(o[2 * dp + 1], pa[kk], b2, b3);
-      }
-    }
-    __syncthreads();  // buffer `buf` is refilled by the next iteration's load
-  }
-  cp_async_wait<0>();
-
-  // ---- finish: O / l, written as (query, head) rows ---------------------------
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f;
-  const float inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
-  T* out = static_cast<T*>(p.out);
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int r = r0 + half * 8;
-    const int i = i0 + r / G;
-    if (i >= C) continue;
-    const float inv = half ? inv1 : inv0;
-    T* orow = out + ((static_cast<int64_t>(b) * C + i) * p.num_q_heads + kvh * G + r % G) * D;
-#pragma unroll
-    for (int n = 0; n < DT; ++n) {
-      const int d = n * 8 + (lane & 3) * 2;
-      const uint32_t v = Mma<T>::pack(o[n][half * 2] * inv, o[n][half * 2 + 1] * inv);
-      *reinterpret_cast<uint32_t*>(orow + d) = v;
-    }
-  }
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
 }
 
 template <typename T, int D, int G>
-int launch(const Params& prm, cudaStream_t s) {
-  constexpr int QT = kBM / G;
-  constexpr int kSmem = kBM * D * 2 + 4 * kBN * D * 2;
-  auto kern = prefill_kernel<T, D, G>;
+int launch(const Params& prm, const void* q, const void* k_cache, const void* v_cache, long long pool_rows,
+           cudaStream_t stream) {
+  constexpr int QT = kM / G;
+  auto enc = encode_fn();
+  if (!enc) return PA_ERR_CUDA;
+  const CUtensorMapDataType dt =
+      Fmt<T>::kCode == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUtensorMap mq, mk, mv;
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(prm.num_q_heads),
+                                static_cast<cuuint64_t>(prm.num_seqs) * prm.chunk};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                   static_cast<cuuint64_t>(prm.num_q_heads) * D * 2};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(QT)};
+    const cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&mq, dt, 3, const_cast<void*>(q), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return PA_ERR_CUDA;
+  }
+  const cuuint64_t kdims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(pool_rows)};
+  const cuuint64_t kstr[1] = {static_cast<cuuint64_t>(D) * 2};
+  const cuuint32_t kbox[2] = {64, static_cast<cuuint32_t>(prm.chunk_rows)};
+  const cuuint32_t kes[2] = {1, 1};
+  if (enc(&mk, dt, 2, const_cast<void*>(k_cache), kdims, kstr, kbox, kes, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return PA_ERR_CUDA;
+  if (enc(&mv, dt, 2, const_cast<void*>(v_cache), kdims, kstr, kbox, kes, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return PA_ERR_CUDA;
+
+  auto kern = prefill_tc_kernel<T, D, G>;
+  // Above half of the SM's shared memory, so one CTA (and one TMEM allocation
+  // of 512 columns) per SM.
+  const int smem = Smem<D>::kAlloc > 120 * 1024 ? Smem<D>::kAlloc : 120 * 1024;
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return PA_ERR_CUDA;
     attr_done[dev] = true;
   }
   dim3 grid((prm.chunk + QT - 1) / QT, prm.num_kv_heads, prm.num_seqs);
-  kern<<<grid, kWarps * 32, kSmem, s>>>(prm);
+  kern<<<grid, kThreads, smem, stream>>>(mq, mk, mv, prm);
   return launch_status();
 }
 
 template <typename T, int D>
-int by_group(const Params& prm, int G, cudaStream_t s) {
+int by_group(const Params& prm, int G, const void* q, const void* k, const void* v, long long rows, cudaStream_t s) {
   switch (G) {
-    case 1: return launch<T, D, 1>(prm, s);
-    case 2: return launch<T, D, 2>(prm, s);
-    case 4: return launch<T, D, 4>(prm, s);
-    case 8: return launch<T, D, 8>(prm, s);
+    case 1: return launch<T, D, 1>(prm, q, k, v, rows, s);
+    case 2: return launch<T, D, 2>(prm, q, k, v, rows, s);
+    case 4: return launch<T, D, 4>(prm, q, k, v, rows, s);
+    case 8: return launch<T, D, 8>(prm, q, k, v, rows, s);
   }
   return PA_ERR_UNSUPPORTED;
 }
 
-template <typename T>
-int by_dim(const Params& prm, int D, int G, cudaStream_t s) {
-  if (D == 64) return by_group<T, 64>(prm, G, s);
-  if (D == 128) return by_group<T, 128>(prm, G, s);
+}  // namespace tc
+
+int prefill_tcgen05(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                    int max_blocks_per_seq, const int32_t* context_lens, int num_seqs, int chunk_len,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                    pa_dtype dtype, cudaStream_t stream) {
+  const long long pool_rows = static_cast<long long>(num_blocks) * num_kv_heads * block_size;
+  if (pool_rows + 16 > 0x7fffffffLL || static_cast<long long>(num_seqs) * chunk_len > 0x7fffffffLL)
+    return PA_ERR_SHAPE;
+  if (!aligned16(out) || (reinterpret_cast<uintptr_t>(q) & 15)) return PA_ERR_ALIGN;
+  tc::Params prm{};
+  prm.out = out;
+  prm.block_tables = block_tables;
+  prm.context_lens = context_lens;
+  prm.err = device_error_word();
+  prm.max_blocks = max_blocks_per_seq;
+  prm.num_seqs = num_seqs;
+  prm.chunk = chunk_len;
+  prm.num_q_heads = num_q_heads;
+  prm.num_kv_heads = num_kv_heads;
+  prm.block_size = block_size;
+  prm.num_blocks = num_blocks;
+  prm.chunk_rows = block_size < 16 ? block_size : 16;
+  prm.oob_row = static_cast<int>(pool_rows);  // first row past the pool: TMA reads zeros
+  prm.scale_log2 = scale * tc::kLog2e;
+  const int G = num_q_heads / num_kv_heads;
+  if (dtype == PA_BF16) {
+    if (head_dim == 128) return tc::by_group<__nv_bfloat16, 128>(prm, G, q, k_cache, v_cache, pool_rows, stream);
+    if (head_dim == 64) return tc::by_group<__nv_bfloat16, 64>(prm, G, q, k_cache, v_cache, pool_rows, stream);
+  } else if (dtype == PA_F16) {
+    if (head_dim == 128) return tc::by_group<__half, 128>(prm, G, q, k_cache, v_cache, pool_rows, stream);
+    if (head_dim == 64) return tc::by_group<__half, 64>(prm, G, q, k_cache, v_cache, pool_rows, stream);
+  }
   return PA_ERR_UNSUPPORTED;
 }
 
-}  // namespace prefill
 }  // namespace pa
 
 using namespace pa;
@@ -370,23 +645,7 @@ extern "C" PA_API int pa_prefill_chunk(void* out, const void* q, const void* k_c
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_NULL;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return PA_ERR_ALIGN;
   if (num_seqs > 65535 || num_kv_heads > 65535) return PA_ERR_SHAPE;
-  prefill::Params prm{};
-  prm.out = out;
-  prm.q = q;
-  prm.k_cache = k_cache;
-  prm.v_cache = v_cache;
-  prm.block_tables = block_tables;
-  prm.context_lens = context_lens;
-  prm.err = device_error_word();
-  prm.max_blocks = max_blocks_per_seq;
-  prm.num_seqs = num_seqs;
-  prm.chunk = chunk_len;
-  prm.num_q_heads = num_q_heads;
-  prm.num_kv_heads = num_kv_heads;
-  prm.block_size = block_size;
-  prm.num_blocks = num_blocks;
-  prm.scale_log2 = scale * prefill::kLog2e;
-  cudaStream_t s = (cudaStream_t)stream;
-  if (dtype == PA_BF16) return prefill::by_dim<__nv_bfloat16>(prm, head_dim, G, s);
-  return prefill::by_dim<__half>(prm, head_dim, G, s);
+  return prefill_tcgen05(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                         chunk_len, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, dtype,
+                         (cudaStream_t)stream);
 }
