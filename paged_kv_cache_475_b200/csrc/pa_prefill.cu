@@ -169,6 +169,48 @@ __host__ __device__ constexpr uint32_t idesc_f16(uint32_t fmt, uint32_t b_mn, in
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------------------
+// 2^x for the softmax. The MUFU unit computes one ex2 per lane-cycle on a
+// pipe 8x narrower than the FMA pipe, and the softmax needs one per score, so
+// a share of the exponentials is computed on the FMA pipe instead (the
+// FMA-offload idea published with FlashAttention-4):
+//   x = j + f, j = round(x) by the 1.5 * 2^23 rounding trick, f in [-1/2, 1/2];
+//   2^f ~ c0 + c1 f + c2 f^2 + c3 f^3, coefficients fitted by this library
+//   (weighted least squares on Chebyshev nodes, max relative error 7.5e-5 on
+//   [-1/2, 1/2], far below the rounding of P to bf16/f16);
+//   2^j is added to the exponent field of the result (as in Schraudolph's
+//   exponent-field construction). x is clamped to [-125, 125] so the result
+//   stays a normal float, and anything below -125 (masked scores, -inf)
+//   returns exactly 0 like ex2.approx.ftz does.
+// ---------------------------------------------------------------------------
+#ifndef PA_TC_POLY_OF_4
+#define PA_TC_POLY_OF_4 0  // pairs of scores out of every 4 that take the FMA path (0 measured fastest)
+#endif
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716648042202f;
+
+__device__ inline float ex2_mufu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ inline float ex2_fma(float x) {
+  const bool zero = !(x >= -125.f);
+  x = fminf(fmaxf(x, -125.f), 125.f);
+  const float y = x + 12582912.f;  // 1.5 * 2^23: the low mantissa bits of y hold round(x)
+  const float j = y - 12582912.f;
+  const float f = x - j;
+  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  return zero ? 0.f : __int_as_float(__float_as_int(p) + (__float_as_int(y) << 23));
+}
+template <bool kFma>
+__device__ inline float ex2_sel(float x) {
+  if constexpr (kFma) return ex2_fma(x);
+  else return ex2_mufu(x);
+}
+
 template <typename T> struct Fmt;
 template <> struct Fmt<__nv_bfloat16> {
   static constexpr uint32_t kCode = 1;
@@ -427,7 +469,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           const int t = t0 + c * 32 + e;
           const float a0 = (masked_tile && t > pos) ? -INFINITY : v[e];
           const float a1 = (masked_tile && t + 1 > pos) ? -INFINITY : v[e + 1];
-          const uint32_t u = Fmt<T>::pack(exp2f(fmaf(a0, p.scale_log2, -m_sub)), exp2f(fmaf(a1, p.scale_log2, -m_sub)));
+          const float x0 = fmaf(a0, p.scale_log2, -m_sub), x1 = fmaf(a1, p.scale_log2, -m_sub);
+          const bool fma_path = ((e / 2) % 4) < PA_TC_POLY_OF_4;
+          const uint32_t u = fma_path ? Fmt<T>::pack(ex2_sel<true>(x0), ex2_sel<true>(x1))
+                                      : Fmt<T>::pack(ex2_sel<false>(x0), ex2_sel<false>(x1));
           pk[(c * 32 + e) / 2] = u;
           psum += Fmt<T>::sum2(u);
         }
