@@ -235,6 +235,10 @@ PA_API size_t pa_noalloc_scratch_bytes(void);
  */
 PA_API int pa_read_error_flags(uint32_t* host_flags, int clear);
 
+/* Message of the last CUDA failure behind a PA_ERR_CUDA returned on this host
+ * thread (the failing step, CUDA's error string and name); "" if none. */
+PA_API const char* pa_last_cuda_error(void);
+
 /* Human-readable name of a pa_status value. */
 PA_API const char* pa_status_string(int status);
 

@@ -25,6 +25,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 PA_F32, PA_F16, PA_BF16 = 0, 1, 2
+PA_ERR_CUDA = -6
 _DT = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
 
 DEVERR_BLOCK_ID = 0x1
@@ -49,12 +50,14 @@ _SIGS = {
     "pa_noalloc_scratch_bytes": [],
     "pa_read_error_flags": [ctypes.POINTER(ctypes.c_uint32), _i],
     "pa_status_string": [_i],
+    "pa_last_cuda_error": [],
     "pa_version": [],
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(_lib, _name)
     _fn.argtypes = _args
-    _fn.restype = {"pa_status_string": ctypes.c_char_p, "pa_noalloc_scratch_bytes": _sz}.get(_name, _i)
+    _fn.restype = {"pa_status_string": ctypes.c_char_p, "pa_last_cuda_error": ctypes.c_char_p,
+                   "pa_noalloc_scratch_bytes": _sz}.get(_name, _i)
 
 
 class PagedAttentionError(RuntimeError):
@@ -63,7 +66,10 @@ class PagedAttentionError(RuntimeError):
 
 def _check(status: int, name: str) -> None:
     if status != 0:
-        raise PagedAttentionError(f"{name}: {_lib.pa_status_string(status).decode()}")
+        msg = f"{name}: {_lib.pa_status_string(status).decode()}"
+        if status == PA_ERR_CUDA:
+            msg += f" [{_lib.pa_last_cuda_error().decode()}]"
+        raise PagedAttentionError(msg)
 
 
 def _ptr(t: torch.Tensor | None):

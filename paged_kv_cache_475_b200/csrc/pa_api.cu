@@ -1,4 +1,5 @@
 // Library-wide entry points: device error word, status strings, version.
+#include <cstdio>
 #include <mutex>
 
 #include "pa_common.cuh"
@@ -26,7 +27,18 @@ unsigned int* device_error_word() {
   return g_err_ptr[dev];
 }
 
+namespace {
+thread_local char g_last_error[256] = "";
+}
+
+int record_cuda_error(cudaError_t e, const char* where) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorString(e), cudaGetErrorName(e));
+  return PA_ERR_CUDA;
+}
+
 }  // namespace pa
+
+extern "C" PA_API const char* pa_last_cuda_error(void) { return pa::g_last_error; }
 
 extern "C" PA_API int pa_read_error_flags(uint32_t* host_flags, int clear) {
   if (!host_flags) return PA_ERR_NULL;

@@ -25,9 +25,13 @@ inline bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8
 
 inline int dtype_bytes(pa_dtype dt) { return dt == PA_F32 ? 4 : 2; }
 
+// Records the message of the last failing CUDA call of this host thread
+// (read back with pa_last_cuda_error) and maps it to PA_ERR_CUDA.
+int record_cuda_error(cudaError_t e, const char* where);
+
 inline int launch_status() {
   cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return e == cudaSuccess ? PA_OK : record_cuda_error(e, "kernel launch");
 }
 
 // ---------------------------------------------------------------------------

@@ -660,8 +660,8 @@ int launch_decode(const DecodeParams& prm, int grid_x, cudaStream_t stream) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, M::kTotal) != cudaSuccess)
-      return PA_ERR_CUDA;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, M::kTotal);
+    if (e != cudaSuccess) return record_cuda_error(e, "decode: set max dynamic shared memory");
     attr_done[dev] = true;
   }
   dim3 grid(grid_x, prm.num_kv_heads, prm.num_seqs);

@@ -8,18 +8,19 @@
 // PagedAttention" (FlashAttention "Cómo funciona"); key tiles past a query
 // tile are never computed, the causal mask is applied in registers.
 //
-// One CTA (6 warps) per (sequence, KV head, 128-row query tile); the 128 rows
+// One CTA (10 warps) per (sequence, KV head, 128-row query tile); the 128 rows
 // are (query, head) pairs of one GQA group, so each gathered K/V page serves
 // all G heads of the group. Warp roles:
-//   warps 0-3  softmax: thread r owns row r (TMEM lane r); reads its S row
-//              from TMEM, keeps the running max / sum, writes P (bf16/f16) to
-//              shared memory, rescales its O row in TMEM when its max grows by
-//              more than 2^8, and finally writes O / l;
-//   warp 4     producer: TMA tensor copies of the Q tile (once) and of each
+//   warps 0-7  softmax: warps w and w+4 own row block 32*(w%4).. (TMEM lanes)
+//              and each take half of the 128 key columns; they read S from
+//              TMEM once, keep the running max / sum, write P (bf16/f16) to
+//              shared memory, rescale their half of the O row in TMEM when the
+//              max grows by more than 2^8, and finally write O / l;
+//   warp 8     producer: TMA tensor copies of the Q tile (once) and of each
 //              128-key K/V tile, gathered page by page through the block table
 //              (one 2-D box of min(B,16) rows per page chunk, 128-byte swizzle;
 //              chunks past the context read out of range and land as zeros);
-//   warp 5     MMA: one thread issues S = Q K^T into a double-buffered TMEM
+//   warp 9     MMA: one thread issues S = Q K^T into a double-buffered TMEM
 //              accumulator and O += P V into a TMEM accumulator (M = 128,
 //              N = 128, K = 16 per instruction), completions via tcgen05.commit
 //              on mbarriers; it zeroes V rows past the context in the last
@@ -39,7 +40,9 @@ namespace tc {
 constexpr int kM = 128;        // query rows per CTA = TMEM lanes
 constexpr int kN = 128;        // keys per tile
 constexpr int kStages = 2;     // K and V rings
-constexpr int kThreads = 192;  // 4 softmax warps + producer + MMA
+constexpr int kThreads = 320;  // 8 softmax warps + producer + MMA
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;  // keep a stale max until the true one is 2^8 larger
@@ -68,7 +71,9 @@ struct Smem {
   // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full, o_done
   static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2;
   static constexpr int oTmem = oBar + kNumBars * 8;
-  static constexpr int kUsed = oTmem + 16;
+  static constexpr int oRed = oTmem + 16;     // row-max exchange [2 parities][2 halves][128 rows]
+  static constexpr int oSum = oRed + 2048;    // row-sum exchange [2 halves][128 rows]
+  static constexpr int kUsed = oSum + 1024;
   static constexpr int kAlloc = kUsed + 1024;  // room to align the base to 1024 B
 };
 
@@ -92,6 +97,21 @@ __device__ inline void fence_proxy_async_smem() { asm volatile("fence.proxy.asyn
 __device__ inline void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
                : "memory");
+}
+
+// Barrier over `count` threads (whole warps) with id `id`; returns the AND of
+// `pred` over them, so every participant takes the same branch afterwards.
+__device__ inline bool pair_and(int id, int count, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(out)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return out != 0;
 }
 
 __device__ inline void mbar_arrive(uint64_t* bar) {
@@ -221,6 +241,9 @@ template <> struct Fmt<__nv_bfloat16> {
   __device__ static inline float sum2(uint32_t u) {
     return __uint_as_float(u << 16) + __uint_as_float(u & 0xffff0000u);
   }
+  __device__ static inline float2 unpack2(uint32_t u) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+  }
 };
 template <> struct Fmt<__half> {
   static constexpr uint32_t kCode = 0;
@@ -232,6 +255,7 @@ template <> struct Fmt<__half> {
     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u));
     return f.x + f.y;
   }
+  __device__ static inline float2 unpack2(uint32_t u) { return __half22float2(*reinterpret_cast<const __half2*>(&u)); }
 };
 
 // Every wait of this kernel gives up after about 2 s and is made warp-uniform,
@@ -241,6 +265,8 @@ __device__ inline bool wait_all(uint64_t* bar, uint32_t parity) {
 }
 
 template <typename T, int D, int G>
+// 10 warps per CTA: the 4 SM sub-partitions hold 16K registers each and two
+// of them host 3 warps, so 168 registers per thread is the ceiling.
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -292,11 +318,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, 8);
     mbar_init(o_done, 1);
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -309,7 +335,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const uint32_t sQ = sb + S::oQ, sK = sb + S::oK, sV = sb + S::oV, sP = sb + S::oP;
   const int32_t* bt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------ producer ------------------------------
     if (n_tiles > 0) {
       if (lane == 0) {
@@ -359,7 +385,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // -------------------------------- MMA ---------------------------------
     bool ok = n_tiles == 0 || wait_all(q_full, 0);
     auto issue_pv = [&](int k) -> bool {
@@ -422,32 +448,47 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (!ok && lane == 0) set_error(p.err, PA_DEVERR_WAIT);
   } else {
     // ------------------------------ softmax -------------------------------
-    const int r = threadIdx.x;                 // row = TMEM lane
+    // Warps w and w + 4 share TMEM lanes 32*(w%4).. (the rows) and split each
+    // row's 128 key columns in halves; they trade row maxima (and at the end
+    // row sums) through shared memory at a 64-thread barrier that also ANDs
+    // their wait outcomes, so both always take the same branch.
+    constexpr int HC = kN / 2;                 // key columns per half
+    constexpr int HD = D / 2;                  // output columns per half
+    const int quad = warp & 3, half = warp >> 2;
+    const int r = quad * 32 + lane;            // row = TMEM lane
     const int i = i0 + r / G, g = r % G;
     const int pos = L - C + i;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    float m = -INFINITY, l = 0.f;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const int bar_id = 1 + quad;
+    float* red = reinterpret_cast<float*>(smem + S::oRed);
+    float* rsum = reinterpret_cast<float*>(smem + S::oSum);
+    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+    float m = -INFINITY, l = 0.f;              // l: this half's share of the row sum
     bool ok = true;
     for (int j = 0; j < n_tiles && ok; ++j) {
-      ok = wait_all(&s_full[j & 1], (j >> 1) & 1);
-      if (!ok) break;
+      bool got = wait_all(&s_full[j & 1], (j >> 1) & 1);
       tc_fence_after();
-      const uint32_t tS = ((j & 1) ? tS1 : tS0) + lane_off;
-      const int t0 = j * kN;
-      const bool masked_tile = t0 + kN - 1 > pos_lo;
-      // pass 1: row max of the (masked) raw scores
+      float v[HC];
+      if (got) {
+        const uint32_t tS = ((j & 1) ? tS1 : tS0) + lane_off + half * HC;
+        tmem_ld32(tS, v);
+        tmem_ld32(tS + 32, v + 32);
+        tmem_wait_ld();
+      }
+      const int t0 = j * kN + half * HC;       // first key of this half
+      if (j * kN + kN - 1 > pos_lo) {          // diagonal tile: causal mask
+#pragma unroll
+        for (int e = 0; e < HC; ++e)
+          if (t0 + e > pos) v[e] = -INFINITY;
+      }
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kN / 32; ++c) {
-        float v[32];
-        tmem_ld32(tS + c * 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const bool cut = masked_tile && (t0 + c * 32 + e > pos);
-          mx = fmaxf(mx, cut ? -INFINITY : v[e]);
-        }
-      }
+      for (int e = 0; e < HC; ++e) mx = fmaxf(mx, v[e]);
+      float* rb = red + (j & 1) * 256;
+      rb[half * 128 + r] = mx;
+      ok = pair_and(bar_id, 64, got);
+      if (!ok) break;
+      mx = fmaxf(mx, rb[(half ^ 1) * 128 + r]);
       const float m_tile = mx * p.scale_log2;
       const float m_new = fmaxf(m, m_tile);
       // Rescale only when the max grows by more than 2^8 (or on the first
@@ -455,83 +496,80 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const bool rescale = (m == -INFINITY) || (m_new > m + kRescaleLog2);
       const float m_use = rescale ? m_new : m;
       const float m_sub = m_use == -INFINITY ? 0.f : m_use;
-      const float alpha = exp2f(m - m_sub);  // 0 while nothing was seen yet
-      // pass 2: probabilities, packed to the input type
-      uint32_t pk[kN / 2];
-      float psum = 0.f;
+      const float alpha = exp2f(m - m_sub);    // 0 while nothing was seen yet
+      const float2 ms2 = make_float2(-m_sub, -m_sub);
+      uint32_t pk[HC / 2];
+      float2 ps2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < kN / 32; ++c) {
-        float v[32];
-        tmem_ld32(tS + c * 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int t = t0 + c * 32 + e;
-          const float a0 = (masked_tile && t > pos) ? -INFINITY : v[e];
-          const float a1 = (masked_tile && t + 1 > pos) ? -INFINITY : v[e + 1];
-          const float x0 = fmaf(a0, p.scale_log2, -m_sub), x1 = fmaf(a1, p.scale_log2, -m_sub);
-          const bool fma_path = ((e / 2) % 4) < PA_TC_POLY_OF_4;
-          const uint32_t u = fma_path ? Fmt<T>::pack(ex2_sel<true>(x0), ex2_sel<true>(x1))
-                                      : Fmt<T>::pack(ex2_sel<false>(x0), ex2_sel<false>(x1));
-          pk[(c * 32 + e) / 2] = u;
-          psum += Fmt<T>::sum2(u);
-        }
+      for (int e = 0; e < HC; e += 2) {
+        const float2 x = __ffma2_rn(make_float2(v[e], v[e + 1]), sc2, ms2);
+        const bool fma_path = ((e / 2) % 4) < PA_TC_POLY_OF_4;
+        const uint32_t u = fma_path ? Fmt<T>::pack(ex2_sel<true>(x.x), ex2_sel<true>(x.y))
+                                    : Fmt<T>::pack(ex2_sel<false>(x.x), ex2_sel<false>(x.y));
+        pk[e / 2] = u;
+        ps2 = __fadd2_rn(ps2, Fmt<T>::unpack2(u));  // P enters PV rounded; sum the same values
       }
-      l = l * alpha + psum;
+      l = l * alpha + (ps2.x + ps2.y);
       m = m_use;
-      if (j > 0) {  // PV(j-1) must be done before O is touched or P is overwritten
-        ok = wait_all(o_done, (j - 1) & 1);
+      if (j > 0) {  // PV(j-1) must be done before P is overwritten or O is touched
+        got = wait_all(o_done, (j - 1) & 1);
+        ok = pair_and(bar_id, 64, got);
         if (!ok) break;
         tc_fence_after();
+      }
+      // this half's 64 keys of P -> atom `half` of the swizzled K-major P tile
+#pragma unroll
+      for (int c = 0; c < HC / 8; ++c) {
+        const uint32_t off = half * (kM * 128) + (r / 8) * 1024 + (r % 8) * 128 + ((c ^ (r % 8)) * 16);
+        *reinterpret_cast<uint4*>(smem + S::oP + off) =
+            make_uint4(pk[c * 4 + 0], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
+      }
+      if (j > 0) {
         // tcgen05.ld/st are warp-collective: the whole warp takes this branch
         // when any of its rows needs a rescale (the others multiply by 1).
         const bool need = rescale && alpha != 1.f;
         if (__any_sync(0xffffffffu, need)) {
           const float f = need ? alpha : 1.f;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < HD / 32; ++c) {
             float o[32];
-            tmem_ld32(tO + lane_off + c * 32, o);
+            tmem_ld32(tO + lane_off + half * HD + c * 32, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] *= f;
-            tmem_st32(tO + lane_off + c * 32, o);
+            tmem_st32(tO + lane_off + half * HD + c * 32, o);
           }
           tmem_wait_st();
         }
-      }
-      // P row -> shared memory, 128-byte swizzled K-major (2 atoms of 64 keys)
-#pragma unroll
-      for (int c = 0; c < kN / 8; ++c) {
-        const int a = c / 8, cc = c % 8;
-        const uint32_t off = a * (kM * 128) + (r / 8) * 1024 + (r % 8) * 128 + ((cc ^ (r % 8)) * 16);
-        *reinterpret_cast<uint4*>(smem + S::oP + off) =
-            make_uint4(pk[c * 4 + 0], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    // epilogue: out = O / l
+    // epilogue: out = O / (l_half0 + l_half1), each half writes its D/2 columns
+    bool got = ok;
     if (ok && n_tiles > 0) {
-      ok = wait_all(o_done, (n_tiles - 1) & 1);
+      got = wait_all(o_done, (n_tiles - 1) & 1);
       tc_fence_after();
     }
+    rsum[half * 128 + r] = l;
+    ok = pair_and(bar_id, 64, got);
     if (!ok) {
-      set_error(p.err, PA_DEVERR_WAIT);
+      if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
     } else {
+      const float lt = l + rsum[(half ^ 1) * 128 + r];
       // Every thread of the warp reads its O row (warp-collective tcgen05.ld);
       // only rows of real queries (i < C) are stored.
       const bool store = i < C;
-      const float inv = (l > 0.f && n_tiles > 0) ? 1.f / l : 0.f;
+      const float inv = (lt > 0.f && n_tiles > 0) ? 1.f / lt : 0.f;
       T* orow = static_cast<T*>(p.out) +
-                ((static_cast<int64_t>(b) * C + (store ? i : 0)) * p.num_q_heads + kvh * G + g) * D;
+                ((static_cast<int64_t>(b) * C + (store ? i : 0)) * p.num_q_heads + kvh * G + g) * D + half * HD;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < HD / 32; ++c) {
         float o[32];
         if (n_tiles > 0) {
-          tmem_ld32(tO + lane_off + c * 32, o);
+          tmem_ld32(tO + lane_off + half * HD + c * 32, o);
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -540,9 +578,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (!store) continue;
 #pragma unroll
         for (int e = 0; e < 32; e += 8) {
-          uint4 v = make_uint4(Fmt<T>::pack(o[e] * inv, o[e + 1] * inv), Fmt<T>::pack(o[e + 2] * inv, o[e + 3] * inv),
+          uint4 w = make_uint4(Fmt<T>::pack(o[e] * inv, o[e + 1] * inv), Fmt<T>::pack(o[e + 2] * inv, o[e + 3] * inv),
                                Fmt<T>::pack(o[e + 4] * inv, o[e + 5] * inv), Fmt<T>::pack(o[e + 6] * inv, o[e + 7] * inv));
-          *reinterpret_cast<uint4*>(orow + c * 32 + e) = v;
+          *reinterpret_cast<uint4*>(orow + c * 32 + e) = w;
         }
       }
     }
@@ -551,7 +589,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 // ---------------------------------------------------------------------------
@@ -576,7 +614,7 @@ int launch(const Params& prm, const void* q, const void* k_cache, const void* v_
            cudaStream_t stream) {
   constexpr int QT = kM / G;
   auto enc = encode_fn();
-  if (!enc) return PA_ERR_CUDA;
+  if (!enc) return record_cuda_error(cudaErrorNotSupported, "prefill: cuTensorMapEncodeTiled unavailable");
   const CUtensorMapDataType dt =
       Fmt<T>::kCode == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap mq, mk, mv;
@@ -590,7 +628,7 @@ int launch(const Params& prm, const void* q, const void* k_cache, const void* v_
     if (enc(&mq, dt, 3, const_cast<void*>(q), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return PA_ERR_CUDA;
+      return record_cuda_error(cudaErrorInvalidValue, "prefill: encode q tensor map");
   }
   const cuuint64_t kdims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(pool_rows)};
   const cuuint64_t kstr[1] = {static_cast<cuuint64_t>(D) * 2};
@@ -599,11 +637,11 @@ int launch(const Params& prm, const void* q, const void* k_cache, const void* v_
   if (enc(&mk, dt, 2, const_cast<void*>(k_cache), kdims, kstr, kbox, kes, CU_TENSOR_MAP_INTERLEAVE_NONE,
           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return PA_ERR_CUDA;
+    return record_cuda_error(cudaErrorInvalidValue, "prefill: encode k tensor map");
   if (enc(&mv, dt, 2, const_cast<void*>(v_cache), kdims, kstr, kbox, kes, CU_TENSOR_MAP_INTERLEAVE_NONE,
           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return PA_ERR_CUDA;
+    return record_cuda_error(cudaErrorInvalidValue, "prefill: encode v tensor map");
 
   auto kern = prefill_tc_kernel<T, D, G>;
   // Above half of the SM's shared memory, so one CTA (and one TMEM allocation
@@ -613,8 +651,8 @@ int launch(const Params& prm, const void* q, const void* k_cache, const void* v_
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return PA_ERR_CUDA;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return record_cuda_error(e, "prefill: set max dynamic shared memory");
     attr_done[dev] = true;
   }
   dim3 grid((prm.chunk + QT - 1) / QT, prm.num_kv_heads, prm.num_seqs);
