@@ -8,21 +8,24 @@
 // PagedAttention" (FlashAttention "Cómo funciona"); key tiles past a query
 // tile are never computed, the causal mask is applied in registers.
 //
-// One CTA (10 warps) per (sequence, KV head, 128-row query tile); the 128 rows
+// One CTA (11 warps) per (sequence, KV head, 128-row query tile); the 128 rows
 // are (query, head) pairs of one GQA group, so each gathered K/V page serves
 // all G heads of the group. Warp roles:
-//   warps 0-7  softmax: warps w and w+4 own row block 32*(w%4).. (TMEM lanes)
-//              and each take half of the 128 key columns; they read S from
-//              TMEM once, keep the running max / sum, write P (bf16/f16) to
-//              shared memory, rescale their half of the O row in TMEM when the
-//              max grows by more than 2^8, and finally write O / l;
-//   warp 8     producer: TMA tensor copies of the Q tile (once) and of each
-//              128-key K/V tile, gathered page by page through the block table
-//              (one 2-D box of min(B,16) rows per page chunk, 128-byte swizzle;
-//              chunks past the context read out of range and land as zeros);
+//   warps 0-7  softmax: warps w and w+4 own row block 32*(w%4).. (TMEM lanes);
+//              warp half h takes keys [64h, 64h+64) of every tile as its own
+//              online-softmax stream (own running max / sum, own TMEM O
+//              accumulator), writes its P (bf16/f16) to shared memory,
+//              rescales its O when its max grows by more than 2^8; the two
+//              streams are joined by the log-sum-exp rule when O is written;
+//   warps 8,10 producers: TMA tensor copies of the Q tile (once) and of each
+//              128-key K tile (warp 8) and V tile (warp 10, its own ring, so a K
+//              load never waits for a V slot), gathered page by page through
+//              the block table (one 2-D box of min(B,16) rows per page chunk,
+//              128-byte swizzle; chunks past the context read out of range
+//              and land as zeros);
 //   warp 9     MMA: one thread issues S = Q K^T into a double-buffered TMEM
-//              accumulator and O += P V into a TMEM accumulator (M = 128,
-//              N = 128, K = 16 per instruction), completions via tcgen05.commit
+//              accumulator and O_h += P_h V_h per key half into two TMEM
+//              accumulators (M = 128, K = 16 per instruction), completions via tcgen05.commit
 //              on mbarriers; it zeroes V rows past the context in the last
 //              partial page chunk before they reach the PV product.
 // Every mbarrier wait is bounded; a timeout sets PA_DEVERR_WAIT and the CTA
@@ -40,9 +43,10 @@ namespace tc {
 constexpr int kM = 128;        // query rows per CTA = TMEM lanes
 constexpr int kN = 128;        // keys per tile
 constexpr int kStages = 2;     // K and V rings
-constexpr int kThreads = 320;  // 8 softmax warps + producer + MMA
-constexpr int kProducerWarp = 8;
+constexpr int kThreads = 352;  // 8 softmax warps + K producer + MMA + V producer
+constexpr int kProducerWarp = 8;   // Q once, then K tiles
 constexpr int kMmaWarp = 9;
+constexpr int kVProducerWarp = 10;  // V tiles
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;  // keep a stale max until the true one is 2^8 larger
@@ -68,8 +72,8 @@ struct Smem {
   static constexpr int oV = oK + kStages * kKV;
   static constexpr int oP = oV + kStages * kKV;
   static constexpr int oBar = oP + kP;
-  // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full, o_done
-  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2;
+  // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_done[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2;
   static constexpr int oTmem = oBar + kNumBars * 8;
   static constexpr int oRed = oTmem + 16;     // row-max exchange [2 parities][2 halves][128 rows]
   static constexpr int oSum = oRed + 2048;    // row-sum exchange [2 halves][128 rows]
@@ -232,9 +236,27 @@ __device__ inline float ex2_sel(float x) {
 }
 
 template <typename T> struct Fmt;
+#ifndef PA_TC_INT_PACK
+#define PA_TC_INT_PACK 0  // the cvt pack measured faster (624 vs 601 TFLOP/s)
+#endif
 template <> struct Fmt<__nv_bfloat16> {
   static constexpr uint32_t kCode = 1;
   __device__ static inline uint32_t pack(float x, float y) {
+#if PA_TC_INT_PACK
+    // Round-to-nearest-even to bf16 with integer ops (ALU pipe, keeping the
+    // conversion off the MUFU/XU pipe that the exponentials saturate). Valid
+    // for the finite, non-negative probabilities this is used on.
+    uint32_t ux = __float_as_uint(x), uy = __float_as_uint(y);
+    ux += 0x7fffu + ((ux >> 16) & 1u);
+    uy += 0x7fffu + ((uy >> 16) & 1u);
+    return __byte_perm(ux, uy, 0x7632);
+#else
+    __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+    return *reinterpret_cast<uint32_t*>(&h);
+#endif
+  }
+  // Round-to-nearest-even of any fp32 pair (used for the output rows).
+  __device__ static inline uint32_t pack_any(float x, float y) {
     __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
     return *reinterpret_cast<uint32_t*>(&h);
   }
@@ -251,6 +273,7 @@ template <> struct Fmt<__half> {
     __half2 h = __floats2half2_rn(x, y);
     return *reinterpret_cast<uint32_t*>(&h);
   }
+  __device__ static inline uint32_t pack_any(float x, float y) { return pack(x, y); }
   __device__ static inline float sum2(uint32_t u) {
     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u));
     return f.x + f.y;
@@ -265,8 +288,8 @@ __device__ inline bool wait_all(uint64_t* bar, uint32_t parity) {
 }
 
 template <typename T, int D, int G>
-// 10 warps per CTA: the 4 SM sub-partitions hold 16K registers each and two
-// of them host 3 warps, so 168 registers per thread is the ceiling.
+// 11 warps per CTA: the 4 SM sub-partitions hold 16K registers each and
+// three of them host 3 warps, so 168 registers per thread is the ceiling.
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -288,8 +311,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   uint64_t* v_full = k_empty + kStages;
   uint64_t* v_empty = v_full + kStages;
   uint64_t* s_full = v_empty + kStages;   // [2]
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = p_full + 1;
+  uint64_t* p_full = s_full + 2;  // [2]: one per key half
+  uint64_t* o_done = p_full + 2;  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::oTmem);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -318,8 +341,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
-    mbar_init(p_full, 8);
-    mbar_init(o_done, 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&p_full[h], 4);
+      mbar_init(&o_done[h], 1);
+    }
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -330,69 +355,65 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS0 = tmem, tS1 = tmem + kN, tO = tmem + 2 * kN;
+  // TMEM columns: S (double buffer) [0, 256), O of key half 0 [256, 256 + D),
+  // O of key half 1 [256 + D, 256 + 2D).
+  const uint32_t tS0 = tmem, tS1 = tmem + kN;
+  const uint32_t tO0 = tmem + 2 * kN, tO1 = tmem + 2 * kN + D;
 
   const uint32_t sQ = sb + S::oQ, sK = sb + S::oK, sV = sb + S::oV, sP = sb + S::oP;
   const int32_t* bt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
 
-  if (warp == kProducerWarp) {
-    // ------------------------------ producer ------------------------------
+  if (warp == kProducerWarp || warp == kVProducerWarp) {
+    // ------------------------- producers (K and V) -------------------------
+    // One warp per ring, so a K tile never waits for a V slot to free up.
+    const bool is_k = warp == kProducerWarp;
     if (n_tiles > 0) {
-      if (lane == 0) {
+      if (is_k && lane == 0) {
         mbar_arrive_expect_tx(q_full, S::kQ);
         for (int a = 0; a < KA; ++a)
           tma_load_3d(sQ + a * (kM * 128), &tm_q, a * 64, kvh * G, b * C + i0, q_full);
       }
       const int R = p.chunk_rows;
       const int chunks = kN / R;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+      const uint32_t ring = is_k ? sK : sV;
       for (int j = 0; j < n_tiles; ++j) {
         const int st = j % kStages;
-        const uint32_t par = ((j / kStages) & 1) ^ 1;
-        bool ok = wait_all(&k_empty[st], par);
-        if (lane == 0) mbar_arrive_expect_tx(&k_full[st], S::kKV);
+        if (!wait_all(&empty[st], ((j / kStages) & 1) ^ 1)) {
+          if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
+          break;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], S::kKV);
         __syncwarp();
         // lane c gathers page chunk c (and c + 32 when B = 8) of this tile
-        int ys[2] = {p.oob_row, p.oob_row};
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int c = lane + 32 * u;
           if (c < chunks) {
             const int t0 = j * kN + c * R;
+            int y = p.oob_row;  // chunks past the context read out of range: zeros
             if (t0 < L) {
               const int id = bt[t0 / B];
               if (id >= 0 && id < p.num_blocks)
-                ys[u] = (id * p.num_kv_heads + kvh) * B + (t0 % B);
+                y = (id * p.num_kv_heads + kvh) * B + (t0 % B);
               else
                 set_error(p.err, PA_DEVERR_BLOCK_ID);
             }
             for (int a = 0; a < KA; ++a)
-              tma_load_2d(sK + st * S::kKV + a * (kN * 128) + c * R * 128, &tm_k, a * 64, ys[u], &k_full[st]);
+              tma_load_2d(ring + st * S::kKV + a * (kN * 128) + c * R * 128, map, a * 64, y, &full[st]);
           }
-        }
-        ok = wait_all(&v_empty[st], par) && ok;
-        if (lane == 0) mbar_arrive_expect_tx(&v_full[st], S::kKV);
-        __syncwarp();
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int c = lane + 32 * u;
-          if (c < chunks)
-            for (int a = 0; a < KA; ++a)
-              tma_load_2d(sV + st * S::kKV + a * (kN * 128) + c * R * 128, &tm_v, a * 64, ys[u], &v_full[st]);
-        }
-        if (!ok) {
-          if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
-          break;
         }
       }
     }
   } else if (warp == kMmaWarp) {
     // -------------------------------- MMA ---------------------------------
     bool ok = n_tiles == 0 || wait_all(q_full, 0);
+    // PV of tile k, one key half at a time: O_h += P[:, half h] V[half h, :].
     auto issue_pv = [&](int k) -> bool {
       const int st = k % kStages;
-      bool good = wait_all(p_full, k & 1);
-      good = wait_all(&v_full[st], (k / kStages) & 1) && good;
-      if (!good) return false;
+      if (!wait_all(&v_full[st], (k / kStages) & 1)) return false;
       // V rows past the context inside the last page chunk hold whatever the
       // pool holds there; P is 0 for them but 0 * NaN is NaN, so zero them.
       const int R = p.chunk_rows;
@@ -409,18 +430,22 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         fence_proxy_async_smem();
       }
       __syncwarp();
-      tc_fence_after();
-      if (lane == 0) {
 #pragma unroll
-        for (int kk = 0; kk < kN / 16; ++kk) {
-          const uint64_t ad = sw128_desc(sP + (kk / 4) * (kM * 128) + (kk % 4) * 32, 1, 64);
-          const uint64_t bd = sw128_desc(sV + st * S::kKV + kk * 2048, (kN * 128) >> 4, 64);
-          tc_mma(tO, ad, bd, kIdescO, (k > 0 || kk > 0) ? 1u : 0u);
+      for (int h = 0; h < 2; ++h) {
+        if (!wait_all(&p_full[h], k & 1)) return false;
+        tc_fence_after();
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
+            const uint64_t ad = sw128_desc(sP + h * (kM * 128) + (kk % 4) * 32, 1, 64);
+            const uint64_t bd = sw128_desc(sV + st * S::kKV + kk * 2048, (kN * 128) >> 4, 64);
+            tc_mma(h ? tO1 : tO0, ad, bd, kIdescO, (k > 0 || kk > 4 * h) ? 1u : 0u);
+          }
+          tc_commit(&o_done[h]);
+          if (h == 1) tc_commit(&v_empty[st]);
         }
-        tc_commit(o_done);
-        tc_commit(&v_empty[st]);
+        __syncwarp();
       }
-      __syncwarp();
       return true;
     };
     for (int j = 0; j < n_tiles && ok; ++j) {
@@ -448,12 +473,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (!ok && lane == 0) set_error(p.err, PA_DEVERR_WAIT);
   } else {
     // ------------------------------ softmax -------------------------------
-    // Warps w and w + 4 share TMEM lanes 32*(w%4).. (the rows) and split each
-    // row's 128 key columns in halves; they trade row maxima (and at the end
-    // row sums) through shared memory at a 64-thread barrier that also ANDs
-    // their wait outcomes, so both always take the same branch.
+    // Warps w and w + 4 share TMEM lanes 32*(w%4).. (the rows). Warp half h
+    // takes keys [64h, 64h + 64) of every tile and runs its own online softmax
+    // over them (own running max / sum, own O accumulator, own P-ready and
+    // PV-done barriers), so the halves never wait for each other inside the
+    // loop; the epilogue joins the two streams with the log-sum-exp rule.
     constexpr int HC = kN / 2;                 // key columns per half
-    constexpr int HD = D / 2;                  // output columns per half
+    constexpr int HD = D / 2;                  // output columns each half writes
     const int quad = warp & 3, half = warp >> 2;
     const int r = quad * 32 + lane;            // row = TMEM lane
     const int i = i0 + r / G, g = r % G;
@@ -463,32 +489,36 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     float* red = reinterpret_cast<float*>(smem + S::oRed);
     float* rsum = reinterpret_cast<float*>(smem + S::oSum);
     const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-    float m = -INFINITY, l = 0.f;              // l: this half's share of the row sum
+    const uint32_t tO = (half ? tO1 : tO0) + lane_off;
+    float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_tiles && ok; ++j) {
-      bool got = wait_all(&s_full[j & 1], (j >> 1) & 1);
+    for (int j = 0; j < n_tiles; ++j) {
+      if (!wait_all(&s_full[j & 1], (j >> 1) & 1)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       float v[HC];
-      if (got) {
+      {
         const uint32_t tS = ((j & 1) ? tS1 : tS0) + lane_off + half * HC;
         tmem_ld32(tS, v);
         tmem_ld32(tS + 32, v + 32);
         tmem_wait_ld();
       }
       const int t0 = j * kN + half * HC;       // first key of this half
-      if (j * kN + kN - 1 > pos_lo) {          // diagonal tile: causal mask
+      if (t0 + HC - 1 > pos_lo) {              // causal mask on the diagonal
 #pragma unroll
         for (int e = 0; e < HC; ++e)
           if (t0 + e > pos) v[e] = -INFINITY;
       }
-      float mx = -INFINITY;
+      float mx8[8];
 #pragma unroll
-      for (int e = 0; e < HC; ++e) mx = fmaxf(mx, v[e]);
-      float* rb = red + (j & 1) * 256;
-      rb[half * 128 + r] = mx;
-      ok = pair_and(bar_id, 64, got);
-      if (!ok) break;
-      mx = fmaxf(mx, rb[(half ^ 1) * 128 + r]);
+      for (int k = 0; k < 8; ++k) mx8[k] = v[k];
+#pragma unroll
+      for (int e = 8; e < HC; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], v[e]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + 4]);
+      const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
       const float m_tile = mx * p.scale_log2;
       const float m_new = fmaxf(m, m_tile);
       // Rescale only when the max grows by more than 2^8 (or on the first
@@ -499,7 +529,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float alpha = exp2f(m - m_sub);    // 0 while nothing was seen yet
       const float2 ms2 = make_float2(-m_sub, -m_sub);
       uint32_t pk[HC / 2];
-      float2 ps2 = make_float2(0.f, 0.f);
+      float2 ps2[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) ps2[k] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int e = 0; e < HC; e += 2) {
         const float2 x = __ffma2_rn(make_float2(v[e], v[e + 1]), sc2, ms2);
@@ -507,17 +539,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint32_t u = fma_path ? Fmt<T>::pack(ex2_sel<true>(x.x), ex2_sel<true>(x.y))
                                     : Fmt<T>::pack(ex2_sel<false>(x.x), ex2_sel<false>(x.y));
         pk[e / 2] = u;
-        ps2 = __fadd2_rn(ps2, Fmt<T>::unpack2(u));  // P enters PV rounded; sum the same values
+        ps2[(e / 2) & 3] = __fadd2_rn(ps2[(e / 2) & 3], Fmt<T>::unpack2(u));  // sum of the rounded P
       }
-      l = l * alpha + (ps2.x + ps2.y);
+      const float2 pa2 = __fadd2_rn(__fadd2_rn(ps2[0], ps2[1]), __fadd2_rn(ps2[2], ps2[3]));
+      l = l * alpha + (pa2.x + pa2.y);
       m = m_use;
-      if (j > 0) {  // PV(j-1) must be done before P is overwritten or O is touched
-        got = wait_all(o_done, (j - 1) & 1);
-        ok = pair_and(bar_id, 64, got);
-        if (!ok) break;
+      if (j > 0) {  // PV(j-1) of this half must be done before P is overwritten or O touched
+        if (!wait_all(&o_done[half], (j - 1) & 1)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
       }
-      // this half's 64 keys of P -> atom `half` of the swizzled K-major P tile
 #pragma unroll
       for (int c = 0; c < HC / 8; ++c) {
         const uint32_t off = half * (kM * 128) + (r / 8) * 1024 + (r % 8) * 128 + ((c ^ (r % 8)) * 16);
@@ -531,13 +564,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (__any_sync(0xffffffffu, need)) {
           const float f = need ? alpha : 1.f;
 #pragma unroll
-          for (int c = 0; c < HD / 32; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             float o[32];
-            tmem_ld32(tO + lane_off + half * HD + c * 32, o);
+            tmem_ld32(tO + c * 32, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] *= f;
-            tmem_st32(tO + lane_off + half * HD + c * 32, o);
+            tmem_st32(tO + c * 32, o);
           }
           tmem_wait_st();
         }
@@ -545,41 +578,50 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[half]);
     }
-    // epilogue: out = O / (l_half0 + l_half1), each half writes its D/2 columns
+    // epilogue: join the two halves, out = (O0 f0 + O1 f1) / (l0 f0 + l1 f1)
     bool got = ok;
     if (ok && n_tiles > 0) {
-      got = wait_all(o_done, (n_tiles - 1) & 1);
+      got = wait_all(&o_done[half], (n_tiles - 1) & 1);
       tc_fence_after();
     }
+    red[half * 128 + r] = m;
     rsum[half * 128 + r] = l;
     ok = pair_and(bar_id, 64, got);
     if (!ok) {
       if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
     } else {
-      const float lt = l + rsum[(half ^ 1) * 128 + r];
-      // Every thread of the warp reads its O row (warp-collective tcgen05.ld);
-      // only rows of real queries (i < C) are stored.
+      const float m_o = red[(half ^ 1) * 128 + r], l_o = rsum[(half ^ 1) * 128 + r];
+      const float M = fmaxf(m, m_o);
+      const float Ms = M == -INFINITY ? 0.f : M;
+      const float f_self = exp2f(m - Ms), f_other = exp2f(m_o - Ms);
+      const float den = l * f_self + l_o * f_other;
+      const float f0 = half == 0 ? f_self : f_other, f1 = half == 0 ? f_other : f_self;
+      const float inv = (den > 0.f && n_tiles > 0) ? 1.f / den : 0.f;
+      // Every thread reads its O rows (warp-collective tcgen05.ld); only
+      // rows of real queries (i < C) are stored.
       const bool store = i < C;
-      const float inv = (lt > 0.f && n_tiles > 0) ? 1.f / lt : 0.f;
       T* orow = static_cast<T*>(p.out) +
                 ((static_cast<int64_t>(b) * C + (store ? i : 0)) * p.num_q_heads + kvh * G + g) * D + half * HD;
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
-        float o[32];
+        float o[32], o1[32];
         if (n_tiles > 0) {
-          tmem_ld32(tO + lane_off + half * HD + c * 32, o);
+          tmem_ld32(tO0 + lane_off + half * HD + c * 32, o);
+          tmem_ld32(tO1 + lane_off + half * HD + c * 32, o1);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0.f;
+          for (int e = 0; e < 32; ++e) o[e] = o1[e] = 0.f;
         }
         if (!store) continue;
 #pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = (o[e] * f0 + o1[e] * f1) * inv;
+#pragma unroll
         for (int e = 0; e < 32; e += 8) {
-          uint4 w = make_uint4(Fmt<T>::pack(o[e] * inv, o[e + 1] * inv), Fmt<T>::pack(o[e + 2] * inv, o[e + 3] * inv),
-                               Fmt<T>::pack(o[e + 4] * inv, o[e + 5] * inv), Fmt<T>::pack(o[e + 6] * inv, o[e + 7] * inv));
+          uint4 w = make_uint4(Fmt<T>::pack_any(o[e], o[e + 1]), Fmt<T>::pack_any(o[e + 2], o[e + 3]),
+                               Fmt<T>::pack_any(o[e + 4], o[e + 5]), Fmt<T>::pack_any(o[e + 6], o[e + 7]));
           *reinterpret_cast<uint4*>(orow + c * 32 + e) = w;
         }
       }
