@@ -42,7 +42,14 @@ namespace tc {
 
 constexpr int kM = 128;        // query rows per CTA = TMEM lanes
 constexpr int kN = 128;        // keys per tile
-constexpr int kStages = 2;     // K and V rings
+#ifndef PA_TC_KSTAGES
+#define PA_TC_KSTAGES 2  // 3 measured slower (smaller L1 carve-out)
+#endif
+#ifndef PA_TC_BT_PREFETCH
+#define PA_TC_BT_PREFETCH 0  // no measurable gain
+#endif
+constexpr int kStagesK = PA_TC_KSTAGES;  // K ring (S = Q K^T needs K earliest)
+constexpr int kStagesV = 2;    // V ring
 constexpr int kThreads = 352;  // 8 softmax warps + K producer + MMA + V producer
 constexpr int kProducerWarp = 8;   // Q once, then K tiles
 constexpr int kMmaWarp = 9;
@@ -69,15 +76,17 @@ struct Smem {
   static constexpr int kP = kM * kN * 2;  // two atoms of [128 rows x 128 B]
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + kQ;
-  static constexpr int oV = oK + kStages * kKV;
-  static constexpr int oP = oV + kStages * kKV;
+  static constexpr int oV = oK + kStagesK * kKV;
+  static constexpr int oP = oV + kStagesV * kKV;
   static constexpr int oBar = oP + kP;
-  // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_done[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2;
+  // q_full, k_full/k_empty[SK], v_full/v_empty[SV], s_full[2], p_full[2], o_done[2]
+  static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 2 + 2 + 2;
   static constexpr int oTmem = oBar + kNumBars * 8;
-  static constexpr int oRed = oTmem + 16;     // row-max exchange [2 parities][2 halves][128 rows]
-  static constexpr int oSum = oRed + 2048;    // row-sum exchange [2 halves][128 rows]
-  static constexpr int kUsed = oSum + 1024;
+  // The epilogue's row-max / row-sum exchange reuses the Q tile, which no
+  // MMA reads any more by then: [2 halves][128 rows] floats each.
+  static constexpr int oRed = oQ;
+  static constexpr int oSum = oQ + 1024;
+  static constexpr int kUsed = oTmem + 16;
   static constexpr int kAlloc = kUsed + 1024;  // room to align the base to 1024 B
 };
 
@@ -307,10 +316,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::oBar);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = k_full + kStages;
-  uint64_t* v_full = k_empty + kStages;
-  uint64_t* v_empty = v_full + kStages;
-  uint64_t* s_full = v_empty + kStages;   // [2]
+  uint64_t* k_empty = k_full + kStagesK;
+  uint64_t* v_full = k_empty + kStagesK;
+  uint64_t* v_empty = v_full + kStagesV;
+  uint64_t* s_full = v_empty + kStagesV;  // [2]
   uint64_t* p_full = s_full + 2;  // [2]: one per key half
   uint64_t* o_done = p_full + 2;  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::oTmem);
@@ -333,9 +342,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStagesK; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < kStagesV; ++s) {
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
@@ -375,36 +386,50 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       const int R = p.chunk_rows;
       const int chunks = kN / R;
+      const int stages = is_k ? kStagesK : kStagesV;
       uint64_t* full = is_k ? k_full : v_full;
       uint64_t* empty = is_k ? k_empty : v_empty;
       const CUtensorMap* map = is_k ? &tm_k : &tm_v;
       const uint32_t ring = is_k ? sK : sV;
-      for (int j = 0; j < n_tiles; ++j) {
-        const int st = j % kStages;
-        if (!wait_all(&empty[st], ((j / kStages) & 1) ^ 1)) {
-          if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
-          break;
-        }
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], S::kKV);
-        __syncwarp();
-        // lane c gathers page chunk c (and c + 32 when B = 8) of this tile
+      // Row coordinates of this lane's page chunks (c = lane, lane + 32) of
+      // tile j; the block-table reads for tile j + 1 are issued before the
+      // wait for tile j + 1's slot, so their latency hides behind it.
+      auto rows_of = [&](int j, int* y) {
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int c = lane + 32 * u;
-          if (c < chunks) {
-            const int t0 = j * kN + c * R;
-            int y = p.oob_row;  // chunks past the context read out of range: zeros
-            if (t0 < L) {
-              const int id = bt[t0 / B];
-              if (id >= 0 && id < p.num_blocks)
-                y = (id * p.num_kv_heads + kvh) * B + (t0 % B);
-              else
-                set_error(p.err, PA_DEVERR_BLOCK_ID);
-            }
-            for (int a = 0; a < KA; ++a)
-              tma_load_2d(ring + st * S::kKV + a * (kN * 128) + c * R * 128, map, a * 64, y, &full[st]);
+          const int t0 = j * kN + c * R;
+          y[u] = p.oob_row;  // chunks past the context read out of range: zeros
+          if (c < chunks && j < n_tiles && t0 < L) {
+            const int id = bt[t0 / B];
+            if (id >= 0 && id < p.num_blocks)
+              y[u] = (id * p.num_kv_heads + kvh) * B + (t0 % B);
+            else
+              set_error(p.err, PA_DEVERR_BLOCK_ID);
           }
         }
+      };
+      int y_cur[2], y_next[2];
+      rows_of(0, y_cur);
+      for (int j = 0; j < n_tiles; ++j) {
+        const int st = j % stages;
+        if (PA_TC_BT_PREFETCH) rows_of(j + 1, y_next);
+        if (!wait_all(&empty[st], ((j / stages) & 1) ^ 1)) {
+          if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
+          break;
+        }
+        if (!PA_TC_BT_PREFETCH) rows_of(j, y_cur);
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], S::kKV);
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int c = lane + 32 * u;
+          if (c < chunks)
+            for (int a = 0; a < KA; ++a)
+              tma_load_2d(ring + st * S::kKV + a * (kN * 128) + c * R * 128, map, a * 64, y_cur[u], &full[st]);
+        }
+        y_cur[0] = y_next[0];
+        y_cur[1] = y_next[1];
       }
     }
   } else if (warp == kMmaWarp) {
@@ -412,8 +437,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     bool ok = n_tiles == 0 || wait_all(q_full, 0);
     // PV of tile k, one key half at a time: O_h += P[:, half h] V[half h, :].
     auto issue_pv = [&](int k) -> bool {
-      const int st = k % kStages;
-      if (!wait_all(&v_full[st], (k / kStages) & 1)) return false;
+      const int st = k % kStagesV;
+      if (!wait_all(&v_full[st], (k / kStagesV) & 1)) return false;
       // V rows past the context inside the last page chunk hold whatever the
       // pool holds there; P is 0 for them but 0 * NaN is NaN, so zero them.
       const int R = p.chunk_rows;
@@ -449,8 +474,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       return true;
     };
     for (int j = 0; j < n_tiles && ok; ++j) {
-      const int st = j % kStages;
-      ok = wait_all(&k_full[st], (j / kStages) & 1);
+      const int st = j % kStagesK;
+      ok = wait_all(&k_full[st], (j / kStagesK) & 1);
       if (!ok) break;
       tc_fence_after();
       if (lane == 0) {
