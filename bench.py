@@ -364,8 +364,18 @@ def run_ours(args):
     args_step = (batch.q, batch.k_new, batch.v_new, batch.k_cache, batch.v_cache, batch.block_tables,
                  batch.context_lens, batch.new_seq, batch.new_pos, batch.scale)
 
-    # Split the step so that the dominant kernel can be timed on its own stream (the current one).
+    # The step, with CUDA events around the dominant kernel (on the current stream, where it runs).
+    fused = (not prefill) and step.fused
+
     def run_step(ev=None):
+        if fused:
+            if ev is not None:
+                ev[0].record(stream)
+            pa.pa_decode_append(step.out, batch.q, batch.k_new, batch.v_new, batch.k_cache, batch.v_cache,
+                                batch.block_tables, batch.context_lens, batch.scale)
+            if ev is not None:
+                ev[1].record(stream)
+            return
         B = batch.k_cache.shape[2]
         pa.pa_slot_mapping(step.slot_mapping, batch.block_tables, batch.new_seq, batch.new_pos, B)
         pa.pa_reshape_and_cache(batch.k_new, batch.v_new, batch.k_cache, batch.v_cache, step.slot_mapping)
@@ -428,8 +438,8 @@ def run_ours(args):
         units_rank = acct["kv_logical"]
         value = sum_over_ranks(units_rank, world) / (ms_step / 1e3) / 1e9
         unit = "GB/s"
-        kname = "pa_decode_splitkv" if partition else "pa_decode"
-        attend_bytes = acct["attend_unique"]
+        kname = "pa_decode_append" if fused else ("pa_decode_splitkv" if partition else "pa_decode")
+        attend_bytes = acct["attend_unique"] + (acct["append"] if fused else 0)
         achieved = attend_bytes / (kern_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "traffic": kernel_traffic(f"{kname}:{args.workload}:B{args.block_size}"),
@@ -486,7 +496,8 @@ def run_ours(args):
             "config": {
                 "workload": WORKLOAD_DESC[args.workload], "num_seqs": batch.num_seqs, "block_size": batch.block_size,
                 "head_dim": batch.head_dim, "num_q_heads": batch.num_q_heads, "num_kv_heads": batch.num_kv_heads,
-                "partition": partition, "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
+                "partition": partition, "fused_append": fused,
+                "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
                 "kv_bytes_logical_per_rank": acct["kv_logical"], "kv_bytes_unique_per_rank": acct["kv_unique"],
                 "parallelism": f"dp{world} (independent batches per GPU)",
             },

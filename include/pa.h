@@ -137,6 +137,26 @@ PA_API int pa_decode(void* out, const void* q, const void* k_cache, const void* 
                      int num_kv_heads, int head_dim, int block_size, int num_blocks,
                      float scale, pa_dtype dtype, void* stream);
 
+/*
+ * pa_decode_append - pa_decode with the step's cache write folded in.
+ *
+ * For decode steps that append exactly one token per sequence, at position
+ * context_lens[b] - 1: first the token's rows are written into its slot,
+ *   k_cache[phys, h, (L_b-1) % B, :] = k_new[b, h, :]   (same for V, every KV head h,
+ *   phys = block_tables[b][(L_b-1) / B]),
+ * exactly as pa_slot_mapping + pa_reshape_and_cache would ([FvP] 内存管理机制,
+ * [FP] PagedAttention steps 1-3), then the output is pa_decode's. One launch
+ * instead of three: the CTA that reads the newest token's page writes the
+ * row itself before its bulk copies read it. k_new/v_new: [N, Hkv, D].
+ * A bad block id for the newest position skips the write and sets
+ * PA_DEVERR_BLOCK_ID. Its page must not be shared with another sequence.
+ */
+PA_API int pa_decode_append(void* out, const void* q, const void* k_new, const void* v_new,
+                            void* k_cache, void* v_cache, const int32_t* block_tables,
+                            int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                            int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                            int num_blocks, float scale, pa_dtype dtype, void* stream);
+
 /* Number of partitions of `partition_size` tokens a context of
  * max_context_len tokens needs (at least 1). */
 PA_API int pa_splitkv_num_partitions(int max_context_len, int partition_size);

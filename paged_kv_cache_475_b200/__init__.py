@@ -40,6 +40,7 @@ _SIGS = {
     "pa_slot_mapping": [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _vp],
     "pa_reshape_and_cache": [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp],
     "pa_decode": [_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp],
+    "pa_decode_append": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp],
     "pa_splitkv_num_partitions": [_i, _i],
     "pa_decode_splitkv": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                           _i, _vp],
@@ -162,6 +163,23 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float
     _check(_lib.pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                           block_tables.shape[1], _ptr(context_lens), N, q.shape[1], Hkv, D, B, P, float(scale),
                           _dtype_code(q), _stream(stream)), "pa_decode")
+
+
+def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, scale: float,
+                     stream=None):
+    """Write each sequence's newest token (k_new/v_new [N, Hkv, D], position L-1) into its slot, then decode."""
+    _need(q, "q", None, 3)
+    _need(out, "out", q.dtype, 3)
+    P, Hkv, B, D, N = _cache_dims(q, k_cache, v_cache, block_tables, context_lens)
+    for n, t in (("k_new", k_new), ("v_new", v_new)):
+        _need(t, n, q.dtype, 3)
+        if t.shape != (N, Hkv, D):
+            raise ValueError(f"{n} must be [N, Hkv, D]")
+    if q.shape[0] != N or q.shape[2] != D or out.shape != q.shape:
+        raise ValueError("q/out must be [N, Hq, D]")
+    _check(_lib.pa_decode_append(_ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                 _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), N, q.shape[1], Hkv,
+                                 D, B, P, float(scale), _dtype_code(q), _stream(stream)), "pa_decode_append")
 
 
 def pa_decode_splitkv(part_o, part_m, part_l, q, k_cache, v_cache, block_tables, context_lens,

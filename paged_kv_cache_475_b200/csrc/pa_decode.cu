@@ -74,6 +74,8 @@ struct DecodeParams {
   int num_parts;
   int longest_first;         // map CTA z-index r to the r-th longest sequence
   float q_scale;             // scale * log2(e)
+  const void* k_new;         // fused append: [N, Hkv, D] rows of each sequence's newest token, or null
+  const void* v_new;
 };
 
 // Sequence whose context is the r-th longest (ties by index). CTAs are
@@ -244,6 +246,32 @@ decode_kernel(const DecodeParams p) {
   const int32_t* bt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
   const int B = p.block_size;
   const int n_seq_blocks = (L + B - 1) / B;
+
+  // ---- fused append: the CTA whose range holds position L-1 writes the
+  // sequence's newest K/V row (this KV head) into its slot before reading.
+  // Generic stores, then a proxy fence and a CTA barrier, so the bulk copies
+  // issued below (async proxy) see the row.
+  if (p.k_new != nullptr && L > 0 && t_begin <= L - 1 && L - 1 < t_end) {
+    if (warp == 0) {
+      const int pos = L - 1;
+      const int phys = bt[pos / B];
+      if (phys >= 0 && phys < p.num_blocks) {
+        constexpr int kChunks = D * S::kEsz / 16;  // 16-byte pieces of one row
+        const int64_t src = (static_cast<int64_t>(b) * p.num_kv_heads + kvh) * D;
+        const int64_t dst = ((static_cast<int64_t>(phys) * p.num_kv_heads + kvh) * B + pos % B) * D;
+        for (int c = lane; c < 2 * kChunks; c += 32) {
+          const bool is_v = c >= kChunks;
+          const int cc = is_v ? c - kChunks : c;
+          const uint4 val = reinterpret_cast<const uint4*>(static_cast<const T*>(is_v ? p.v_new : p.k_new) + src)[cc];
+          reinterpret_cast<uint4*>(const_cast<T*>(is_v ? vc : kc) + dst)[cc] = val;
+        }
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      } else if (lane == 0) {
+        set_error(p.err, PA_DEVERR_BLOCK_ID);
+      }
+    }
+    __syncthreads();
+  }
   const uint64_t policy = l2_evict_first_policy();
 
   // Block ids of this warp's tiles k = 32*c + lane (two ids per tile when B = 8).
@@ -734,6 +762,38 @@ extern "C" PA_API int pa_decode(void* out, const void* q, const void* k_cache, c
   prm.q = q;
   prm.k_cache = k_cache;
   prm.v_cache = v_cache;
+  prm.block_tables = block_tables;
+  prm.context_lens = context_lens;
+  prm.max_blocks = max_blocks_per_seq;
+  prm.num_seqs = num_seqs;
+  prm.num_q_heads = num_q_heads;
+  prm.num_kv_heads = num_kv_heads;
+  prm.block_size = block_size;
+  prm.num_blocks = num_blocks;
+  prm.partition = 0;
+  prm.num_parts = 1;
+  prm.longest_first = num_seqs > 1 && num_seqs <= PA_DECODE_LPT_MAX_SEQS;
+  return run_decode(prm, head_dim, scale, dtype, 1, (cudaStream_t)stream);
+}
+
+extern "C" PA_API int pa_decode_append(void* out, const void* q, const void* k_new, const void* v_new,
+                                       void* k_cache, void* v_cache, const int32_t* block_tables,
+                                       int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                                       int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                       int num_blocks, float scale, pa_dtype dtype, void* stream) {
+  int st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                             num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, dtype);
+  if (st != PA_OK || num_seqs == 0) return st;
+  if (!out || !k_new || !v_new) return PA_ERR_NULL;
+  if (!aligned16(k_new) || !aligned16(v_new)) return PA_ERR_ALIGN;
+  if (num_seqs > 65535) return PA_ERR_SHAPE;
+  DecodeParams prm{};
+  prm.out = out;
+  prm.q = q;
+  prm.k_cache = k_cache;
+  prm.v_cache = v_cache;
+  prm.k_new = k_new;
+  prm.v_new = v_new;
   prm.block_tables = block_tables;
   prm.context_lens = context_lens;
   prm.max_blocks = max_blocks_per_seq;

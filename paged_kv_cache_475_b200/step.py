@@ -11,8 +11,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (pa_decode, pa_decode_splitkv, pa_merge, pa_prefill_chunk, pa_reshape_and_cache,
-               pa_slot_mapping, pa_splitkv_num_partitions)
+from . import (pa_decode, pa_decode_append, pa_decode_splitkv, pa_merge, pa_prefill_chunk,
+               pa_reshape_and_cache, pa_slot_mapping, pa_splitkv_num_partitions)
 
 NUM_SMS_B200 = 148
 
@@ -33,15 +33,25 @@ def choose_partition(num_seqs: int, num_kv_heads: int, max_context_len: int,
 
 
 class DecodeStep:
-    """Append one token per sequence, then decode-attend over the paged cache."""
+    """Append one token per sequence, then decode-attend over the paged cache.
+
+    fused_append: with no split and exactly one new token per sequence (token b
+    of k_new/v_new is sequence b's newest, at position context_lens[b] - 1),
+    the append is folded into the decode kernel (pa_decode_append: one launch).
+    "auto" picks it whenever those conditions hold by construction.
+    """
 
     def __init__(self, num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
                  max_context_len: int, dtype: torch.dtype, num_new_tokens: int | None = None,
-                 partition: int | None | str = "auto", device="cuda"):
+                 partition: int | None | str = "auto", fused_append: bool | str = "auto", device="cuda"):
         self.N, self.Hq, self.D = num_seqs, num_q_heads, head_dim
         if partition == "auto":
             partition = choose_partition(num_seqs, num_kv_heads, max_context_len)
         self.partition = partition
+        one_per_seq = num_new_tokens is None or num_new_tokens == num_seqs
+        self.fused = (not partition and one_per_seq) if fused_append == "auto" else bool(fused_append)
+        if self.fused and (partition or not one_per_seq):
+            raise ValueError("the fused append needs the single-pass decode and one new token per sequence")
         T = num_seqs if num_new_tokens is None else num_new_tokens
         self.slot_mapping = torch.empty(T, dtype=torch.int64, device=device)
         self.out = torch.empty((num_seqs, num_q_heads, head_dim), dtype=dtype, device=device)
@@ -51,10 +61,13 @@ class DecodeStep:
                                       device=device)
             self.part_m = torch.empty((num_seqs, num_q_heads, self.num_parts), dtype=torch.float32, device=device)
             self.part_l = torch.empty_like(self.part_m)
-        self.launches_per_call = 4 if partition else 3
+        self.launches_per_call = 1 if self.fused else (4 if partition else 3)
 
     def __call__(self, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, new_seq, new_pos,
                  scale: float, stream=None):
+        if self.fused:
+            pa_decode_append(self.out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, scale, stream)
+            return self.out
         B = k_cache.shape[2]
         pa_slot_mapping(self.slot_mapping, block_tables, new_seq, new_pos, B, stream)
         pa_reshape_and_cache(k_new, v_new, k_cache, v_cache, self.slot_mapping, stream)
@@ -86,12 +99,12 @@ class PrefillStep:
         return self.out
 
 
-def run_batch(batch, partition: int | None | str = "auto"):
+def run_batch(batch, partition: int | None | str = "auto", fused_append: bool | str = "auto"):
     """Run one step of a workloads.PagedBatch that lives on the GPU; returns the output tensor."""
     if batch.chunk == 1:
         step = DecodeStep(batch.num_seqs, batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
                           int(batch.context_lens.max().item()) if batch.num_seqs else 1, batch.q.dtype,
-                          num_new_tokens=batch.new_seq.shape[0], partition=partition)
+                          num_new_tokens=batch.new_seq.shape[0], partition=partition, fused_append=fused_append)
     else:
         step = PrefillStep(batch.num_seqs, batch.chunk, batch.num_q_heads, batch.head_dim, batch.q.dtype,
                            num_new_tokens=batch.new_seq.shape[0])

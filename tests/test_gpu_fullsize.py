@@ -27,12 +27,12 @@ def llama():
     return b, ref
 
 
-@pytest.mark.parametrize("partition", ["auto", None, 512])
-def test_llama_decode_full(llama, partition):
+@pytest.mark.parametrize("partition,fused", [("auto", "auto"), (None, False), (512, False)])
+def test_llama_decode_full(llama, partition, fused):
     b, ref = llama
-    out, _, flags = run_gpu(b, partition=partition)
+    out, _, flags = run_gpu(b, partition=partition, fused_append=fused)
     assert flags == 0
-    assert_close(out, ref, "f16", f"llama decode partition={partition}")
+    assert_close(out, ref, "f16", f"llama decode partition={partition} fused={fused}")
 
 
 def test_long_context_sampled():

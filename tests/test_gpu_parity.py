@@ -82,9 +82,24 @@ def test_tiny_fp32_decode():
 def test_decode_grid_f16(D, G, B):
     b = small_batch(seed=D * 1000 + G * 100 + B, D=D, G=G, B=B)
     ref, *_ = oracle.step(b)
-    out, _, flags = run_gpu(b, partition=None)
+    out, _, flags = run_gpu(b, partition=None, fused_append=False)
     assert flags == 0
     assert_close(out, ref, "f16", f"D={D} G={G} B={B}")
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("B", [8, 16, 128])
+def test_decode_append_fused(dtype, B):
+    """pa_decode_append: the cache after the call equals the oracle's append bit for bit, and the
+    output (whose newest token was poisoned before the call) matches the oracle."""
+    b = small_batch(seed=17 + B, dtype=dtype, B=B, lens=(1, 15, 16, 17, 100, 333, 700))
+    ref, kc, vc, _ = oracle.step(b)
+    out, g, flags = run_gpu(b, partition=None, fused_append=True)
+    assert flags == 0
+    assert_close(out, ref, dtype, f"fused append {dtype} B={B}")
+    iv = torch.int32 if dtype == "f32" else torch.int16
+    assert torch.equal(g.k_cache.cpu().view(iv), kc.view(iv))
+    assert torch.equal(g.v_cache.cpu().view(iv), vc.view(iv))
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
