@@ -122,6 +122,25 @@ PA_API int pa_reshape_and_cache(const void* k_new, const void* v_new, void* k_ca
                                 int block_size, pa_dtype dtype, void* stream);
 
 /*
+ * pa_copy_blocks - copy whole blocks (all KV heads, K and V) between pools.
+ *
+ * For each i < num_pairs: dst[dst_block_ids[i]] = src[src_block_ids[i]] in
+ * both the K and the V pool, bits unchanged. Covers the copy-on-write of
+ * [FP] PagedAttention "Cómo funciona" step 4 (dst pool == src pool: a
+ * sequence that diverges inside a shared block gets its own copy) and the
+ * swapping of "Flash Attention vs Paged Attention" 恢复机制对比 (one pool in
+ * pinned host memory, which kernels address directly: swap out = device to
+ * host, swap in = host to device). Pools are [num_blocks, Hkv, B, D] in
+ * `dtype`; the id arrays (int32 [num_pairs]) must be device-accessible.
+ * An id outside its pool skips that pair and sets PA_DEVERR_BLOCK_ID. A
+ * destination that is also a source in the same call gives undefined rows.
+ */
+PA_API int pa_copy_blocks(void* dst_k, void* dst_v, int dst_num_blocks, const void* src_k,
+                          const void* src_v, int src_num_blocks, const int32_t* src_block_ids,
+                          const int32_t* dst_block_ids, int num_pairs, int num_kv_heads,
+                          int head_dim, int block_size, pa_dtype dtype, void* stream);
+
+/*
  * pa_decode - one query token per sequence over its whole paged context.
  *
  * out[b, h, :] = sum_t softmax_t(scale * q[b,h,:] . K_b[t]) V_b[t], t < context_lens[b],

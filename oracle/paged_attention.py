@@ -114,6 +114,22 @@ def reshape_and_cache(k_new, v_new, k_cache, v_cache, slots):
     return kc, vc
 
 
+def copy_blocks(dst_k, dst_v, src_k, src_v, src_ids, dst_ids):
+    """Whole-block copies; returns updated copies of the destination pools.
+
+    [FP] PagedAttention "Cómo funciona" step 4 (copy-on-write of a shared
+    block) and the swapping of [FvP] 恢复机制对比: block dst_ids[i] of the
+    destination pool becomes block src_ids[i] of the source pool, bits
+    unchanged, for K and V.
+    """
+    dk, dv = _cpu(dst_k).clone(), _cpu(dst_v).clone()
+    sk, sv = _cpu(src_k), _cpu(src_v)
+    for s_, d_ in zip(_as_i64(src_ids).tolist(), _as_i64(dst_ids).tolist()):
+        dk[d_] = sk[s_]
+        dv[d_] = sv[s_]
+    return dk, dv
+
+
 # --------------------------------------------------------------------------
 # Gather + textbook attention
 # --------------------------------------------------------------------------

@@ -39,6 +39,7 @@ _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_
 _SIGS = {
     "pa_slot_mapping": [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _vp],
     "pa_reshape_and_cache": [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp],
+    "pa_copy_blocks": [_vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp],
     "pa_decode": [_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp],
     "pa_decode_append": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp],
     "pa_splitkv_num_partitions": [_i, _i],
@@ -137,6 +138,33 @@ def pa_reshape_and_cache(k_new, v_new, k_cache, v_cache, slot_mapping, stream=No
     _check(_lib.pa_reshape_and_cache(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
                                      T, P, Hkv, D, B, _dtype_code(k_cache), _stream(stream)),
            "pa_reshape_and_cache")
+
+
+def pa_copy_blocks(dst_k, dst_v, src_k, src_v, src_block_ids, dst_block_ids, stream=None):
+    """dst[dst_block_ids[i]] = src[src_block_ids[i]] for K and V pools [P, Hkv, B, D].
+
+    Pools may be CUDA tensors or pinned host tensors (device-addressable); the
+    id tensors (int32) likewise. Copy-on-write: dst pools = src pools.
+    """
+    for n, t in (("dst_k", dst_k), ("dst_v", dst_v), ("src_k", src_k), ("src_v", src_v)):
+        if not isinstance(t, torch.Tensor) or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous [P, Hkv, B, D] tensor")
+        if not (t.is_cuda or t.is_pinned()):
+            raise ValueError(f"{n} must be a CUDA tensor or pinned host memory")
+    for n, t in (("src_block_ids", src_block_ids), ("dst_block_ids", dst_block_ids)):
+        if t.dtype != torch.int32 or t.dim() != 1 or not (t.is_cuda or t.is_pinned()):
+            raise ValueError(f"{n} must be int32 [n], on the GPU or pinned")
+    if dst_k.shape[1:] != src_k.shape[1:] or dst_v.shape != dst_k.shape or src_v.shape != src_k.shape:
+        raise ValueError("pool shapes differ")
+    if dst_k.dtype != src_k.dtype:
+        raise ValueError("pool dtypes differ")
+    n = src_block_ids.shape[0]
+    if dst_block_ids.shape[0] != n:
+        raise ValueError("id arrays differ in length")
+    _, Hkv, B, D = src_k.shape
+    _check(_lib.pa_copy_blocks(_ptr(dst_k), _ptr(dst_v), dst_k.shape[0], _ptr(src_k), _ptr(src_v), src_k.shape[0],
+                               _ptr(src_block_ids), _ptr(dst_block_ids), n, Hkv, D, B, _dtype_code(src_k),
+                               _stream(stream)), "pa_copy_blocks")
 
 
 def _cache_dims(q, k_cache, v_cache, block_tables, context_lens):

@@ -99,3 +99,63 @@ extern "C" PA_API int pa_reshape_and_cache(const void* k_new, const void* v_new,
       chunks_per_head, num_kv_heads, block_size, device_error_word());
   return launch_status();
 }
+
+// ---------------------------------------------------------------------------
+// Whole-block copies between pools: copy-on-write and swap.
+//
+// [FP] PagedAttention "Cómo funciona" step 4: sequences sharing a prompt
+// point at the same physical blocks and copy a block only when their contents
+// diverge (copy-on-write); "Flash Attention vs Paged Attention" 恢复机制对比:
+// blocks can be swapped out to host memory and back. Both are the same
+// operation on a list of (source block, destination block) pairs; the two
+// pools may be the same device pool (copy-on-write) or a device pool and a
+// pinned host pool (swap out / swap in), which kernels address directly.
+// ---------------------------------------------------------------------------
+namespace pa {
+
+__global__ void copy_blocks_kernel(uint4* __restrict__ dst_k, uint4* __restrict__ dst_v,
+                                   const uint4* __restrict__ src_k, const uint4* __restrict__ src_v,
+                                   const int32_t* __restrict__ src_ids, const int32_t* __restrict__ dst_ids,
+                                   int num_pairs, int64_t chunks_per_block, int src_blocks, int dst_blocks,
+                                   unsigned int* err) {
+  const int64_t total = static_cast<int64_t>(num_pairs) * chunks_per_block;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int pr = static_cast<int>(i / chunks_per_block);
+    const int64_t c = i % chunks_per_block;
+    const int s = src_ids[pr], d = dst_ids[pr];
+    if (s < 0 || s >= src_blocks || d < 0 || d >= dst_blocks) {
+      if (c == 0) set_error(err, PA_DEVERR_BLOCK_ID);
+      continue;
+    }
+    dst_k[d * chunks_per_block + c] = src_k[s * chunks_per_block + c];
+    dst_v[d * chunks_per_block + c] = src_v[s * chunks_per_block + c];
+  }
+}
+
+}  // namespace pa
+
+extern "C" PA_API int pa_copy_blocks(void* dst_k, void* dst_v, int dst_num_blocks, const void* src_k,
+                                     const void* src_v, int src_num_blocks, const int32_t* src_block_ids,
+                                     const int32_t* dst_block_ids, int num_pairs, int num_kv_heads, int head_dim,
+                                     int block_size, pa_dtype dtype, void* stream) {
+  if (num_pairs < 0 || dst_num_blocks < 0 || src_num_blocks < 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      block_size <= 0)
+    return PA_ERR_SHAPE;
+  if (dtype != PA_F32 && dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_DTYPE;
+  if (num_pairs == 0) return PA_OK;
+  if (!dst_k || !dst_v || !src_k || !src_v || !src_block_ids || !dst_block_ids) return PA_ERR_NULL;
+  if (!aligned16(dst_k) || !aligned16(dst_v) || !aligned16(src_k) || !aligned16(src_v)) return PA_ERR_ALIGN;
+  const int64_t block_bytes = static_cast<int64_t>(num_kv_heads) * block_size * head_dim * dtype_bytes(dtype);
+  if (block_bytes % 16) return PA_ERR_UNSUPPORTED;
+  const int64_t chunks = block_bytes / 16;
+  const int64_t total = chunks * num_pairs;
+  const int threads = 256;
+  const int64_t want = (total + threads - 1) / threads;
+  const int blocks = static_cast<int>(want < 148 * 16 ? want : 148 * 16);
+  copy_blocks_kernel<<<blocks, threads, 0, (cudaStream_t)stream>>>(
+      static_cast<uint4*>(dst_k), static_cast<uint4*>(dst_v), static_cast<const uint4*>(src_k),
+      static_cast<const uint4*>(src_v), src_block_ids, dst_block_ids, num_pairs, chunks, src_num_blocks,
+      dst_num_blocks, device_error_word());
+  return launch_status();
+}

@@ -328,9 +328,25 @@ def pin_bytes_per_token(P=None):
     assert abs(gib - 12.207) < 1e-3 and abs(gib - g["page_quote_gib"]) < 0.7
 
 
+def pin_copy_blocks(P):
+    """Block copies: destination blocks take the source blocks' bits, every other block keeps its own."""
+    gen = torch.Generator().manual_seed(9)
+    sk = torch.randn(6, 2, 4, 8, generator=gen).to(torch.bfloat16)
+    sv = torch.randn(6, 2, 4, 8, generator=gen).to(torch.bfloat16)
+    dk = torch.randn(5, 2, 4, 8, generator=gen).to(torch.bfloat16)
+    dv = torch.randn(5, 2, 4, 8, generator=gen).to(torch.bfloat16)
+    src, dst = [4, 0, 4], [1, 3, 0]
+    ok_, ov_ = P.copy_blocks(dk, dv, sk, sv, src, dst)
+    for s_, d_ in zip(src, dst):
+        assert torch.equal(ok_[d_].view(torch.int16), sk[s_].view(torch.int16))
+        assert torch.equal(ov_[d_].view(torch.int16), sv[s_].view(torch.int16))
+    for d_ in (2, 4):
+        assert torch.equal(ok_[d_].view(torch.int16), dk[d_].view(torch.int16))
+
+
 ALL_PINS = [
     pin_uniform_scores_mean_of_v, pin_dominant_key, pin_single_token, pin_block_permutation,
     pin_shared_vs_private, pin_eq4_block_sums, pin_partials_closed_form, pin_merge_empty,
     pin_torch_sdpa, pin_brute_force, pin_prefill_rows_are_truncated_decodes,
-    pin_page_example_slots, pin_cache_write,
+    pin_page_example_slots, pin_cache_write, pin_copy_blocks,
 ]

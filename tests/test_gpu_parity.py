@@ -299,3 +299,86 @@ def test_prefill_short_context_rows_are_zero():
     assert not ref[: 8 * b.num_q_heads].any()
     got = torch.stack([out[0, i, h].cpu() for (_, i, h) in rows])
     assert_close(got, ref, "bf16", "short context")
+
+
+# ---------------------------------------------------------------------------
+# Whole-block copies: copy-on-write and swap
+# ---------------------------------------------------------------------------
+
+def test_copy_blocks_copy_on_write_in_place():
+    import paged_kv_cache_475_b200 as pa
+    b = small_batch(seed=301, dtype="bf16", lens=(40, 70, 90), poison=None)
+    g = b.to("cuda")
+    src = torch.tensor([int(b.block_tables[0, 0]), int(b.block_tables[1, 2]), 5], dtype=torch.int32)
+    dst = torch.tensor([int(b.k_cache.shape[0]) - 1, int(b.k_cache.shape[0]) - 2, 6], dtype=torch.int32)
+    pa.pa_copy_blocks(g.k_cache, g.v_cache, g.k_cache, g.v_cache, src.cuda(), dst.cuda())
+    torch.cuda.synchronize()
+    kc, vc = oracle.copy_blocks(b.k_cache, b.v_cache, b.k_cache, b.v_cache, src, dst)
+    assert torch.equal(g.k_cache.cpu().view(torch.int16), kc.view(torch.int16))
+    assert torch.equal(g.v_cache.cpu().view(torch.int16), vc.view(torch.int16))
+    assert pa.pa_read_error_flags() == 0
+
+
+def test_copy_blocks_swap_out_and_in_through_pinned_host_memory():
+    import paged_kv_cache_475_b200 as pa
+    b = small_batch(seed=302, dtype="f16", lens=(100, 333), poison=None, pool_factor=2.0)
+    g = b.to("cuda")
+    P = b.k_cache.shape[0]
+    ids = b.block_tables[0, :7].clone()                       # sequence 0's blocks
+    host_k = torch.zeros((8,) + tuple(b.k_cache.shape[1:]), dtype=b.k_cache.dtype).pin_memory()
+    host_v = torch.zeros_like(host_k).pin_memory()
+    slots = torch.arange(7, dtype=torch.int32).pin_memory()
+    pa.pa_copy_blocks(host_k, host_v, g.k_cache, g.v_cache, ids.cuda(), slots)      # swap out
+    torch.cuda.synchronize()
+    hk, hv = oracle.copy_blocks(torch.zeros_like(host_k), torch.zeros_like(host_v), b.k_cache, b.v_cache, ids,
+                                torch.arange(7))
+    assert torch.equal(host_k.view(torch.int16), hk.view(torch.int16))
+    assert torch.equal(host_v.view(torch.int16), hv.view(torch.int16))
+    used = set(b.block_tables[b.block_tables >= 0].tolist())
+    new_ids = torch.tensor([i for i in range(P) if i not in used][:7], dtype=torch.int32)
+    pa.pa_copy_blocks(g.k_cache, g.v_cache, host_k, host_v, slots, new_ids.cuda())  # swap in elsewhere
+    torch.cuda.synchronize()
+    assert torch.equal(g.k_cache[new_ids.long()].cpu().view(torch.int16), b.k_cache[ids.long()].view(torch.int16))
+    # the sequence reads the same context through its updated table
+    ref, *_ = oracle.step(b)
+    g.block_tables[0, :7] = new_ids.cuda()
+    from paged_kv_cache_475_b200.step import run_batch
+    out = run_batch(g, partition=None, fused_append=False).cpu()
+    assert_close(out, ref, "f16", "after swap in")
+    assert pa.pa_read_error_flags() == 0
+
+
+def test_copy_on_write_through_the_block_manager():
+    """Two sequences share a half-full block; the second one's next token triggers a copy."""
+    import paged_kv_cache_475_b200 as pa
+    from paged_kv_cache_475_b200.blocks import BlockManager
+    gen = torch.Generator().manual_seed(303)
+    Hkv, Hq, D, B, P = 2, 8, 128, 16, 12
+    m = BlockManager(P, B)
+    m.allocate(0, 40)
+    m.fork(0, 1)
+    kc = torch.randn(P, Hkv, B, D, generator=gen).half()
+    vc = torch.randn(P, Hkv, B, D, generator=gen).half()
+    slot0, pair0 = m.append_slot(0)   # seq 0: first writer of the shared last block -> copy
+    slot1, pair1 = m.append_slot(1)   # seq 1: now alone in the original block
+    assert pair0 is not None and pair1 is None
+    k_new = torch.randn(2, Hkv, D, generator=gen).half()
+    v_new = torch.randn(2, Hkv, D, generator=gen).half()
+    q = torch.randn(2, Hq, D, generator=gen).half()
+    bt = m.tables_tensor([0, 1])
+    lens = torch.tensor([41, 41], dtype=torch.int32)
+    # oracle: copy, then write both new tokens, then attend
+    okc, ovc = oracle.copy_blocks(kc, vc, kc, vc, [pair0[0]], [pair0[1]])
+    okc, ovc = oracle.reshape_and_cache(k_new, v_new, okc, ovc, [slot0, slot1])
+    ref = oracle.attention(q, okc, ovc, bt, lens, D ** -0.5)
+    # library: pa_copy_blocks, pa_reshape_and_cache, pa_decode
+    gk, gv = kc.cuda(), vc.cuda()
+    pa.pa_copy_blocks(gk, gv, gk, gv, torch.tensor([pair0[0]], dtype=torch.int32).cuda(),
+                      torch.tensor([pair0[1]], dtype=torch.int32).cuda())
+    pa.pa_reshape_and_cache(k_new.cuda(), v_new.cuda(), gk, gv, torch.tensor([slot0, slot1]).cuda())
+    out = torch.empty_like(q).cuda()
+    pa.pa_decode(out, q.cuda(), gk, gv, bt.cuda(), lens.cuda(), D ** -0.5)
+    torch.cuda.synchronize()
+    assert torch.equal(gk.cpu().view(torch.int16), okc.view(torch.int16))
+    assert_close(out.cpu(), ref, "f16", "copy on write")
+    assert pa.pa_read_error_flags() == 0

@@ -98,6 +98,11 @@ def partials_normalised(q, k_cache, v_cache, bt, lens, scale, partition, num_par
 
 
 _orig_partials = P.splitkv_partials
+_orig_copy = P.copy_blocks
+
+
+def copy_blocks_shifted(dst_k, dst_v, src_k, src_v, src_ids, dst_ids):
+    return _orig_copy(dst_k, dst_v, src_k, src_v, [(int(s) + 1) % src_k.shape[0] for s in src_ids], dst_ids)
 
 MUTANTS = {
     "pages_reversed": ("gather_sequence", gather_pages_reversed),
@@ -111,6 +116,7 @@ MUTANTS = {
     "slot_block_offset_swapped": ("slot_mapping", slots_swapped),
     "cache_write_row_off": ("reshape_and_cache", cache_write_row_off),
     "partials_normalised": ("splitkv_partials", partials_normalised),
+    "copy_blocks_source_shifted": ("copy_blocks", copy_blocks_shifted),
 }
 
 
