@@ -356,9 +356,12 @@ def run_ours(args):
         partition = None
     else:
         part = "auto" if args.partition == "auto" else (None if args.partition == "none" else int(args.partition))
+        # chat trace: half the batch shares a 1024-token prompt -> the shared-prefix cascade
+        sp = (batch_cpu.info["shared_prefix_tokens"], batch_cpu.info["shared_group"]) \
+            if args.workload == "chat_trace" and args.partition == "auto" else None
         step = DecodeStep(batch.num_seqs, batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
                           int(batch_cpu.context_lens.max()), batch.q.dtype,
-                          num_new_tokens=batch.new_seq.shape[0], partition=part)
+                          num_new_tokens=batch.new_seq.shape[0], partition=part, shared_prefix=sp)
         partition = step.partition
     stream = torch.cuda.current_stream()
     args_step = (batch.q, batch.k_new, batch.v_new, batch.k_cache, batch.v_cache, batch.block_tables,
@@ -366,8 +369,16 @@ def run_ours(args):
 
     # The step, with CUDA events around the dominant kernel (on the current stream, where it runs).
     fused = (not prefill) and step.fused
+    cascade = (not prefill) and getattr(step, "shared_prefix", None) is not None
 
     def run_step(ev=None):
+        if cascade:
+            if ev is not None:
+                ev[0].record(stream)
+            step(*args_step)
+            if ev is not None:
+                ev[1].record(stream)
+            return
         if fused:
             if ev is not None:
                 ev[0].record(stream)
@@ -438,7 +449,8 @@ def run_ours(args):
         units_rank = acct["kv_logical"]
         value = sum_over_ranks(units_rank, world) / (ms_step / 1e3) / 1e9
         unit = "GB/s"
-        kname = "pa_decode_append" if fused else ("pa_decode_splitkv" if partition else "pa_decode")
+        kname = ("pa_decode_shared_prefix" if cascade else
+                 "pa_decode_append" if fused else ("pa_decode_splitkv" if partition else "pa_decode"))
         attend_bytes = acct["attend_unique"] + (acct["append"] if fused else 0)
         achieved = attend_bytes / (kern_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
@@ -497,6 +509,7 @@ def run_ours(args):
                 "workload": WORKLOAD_DESC[args.workload], "num_seqs": batch.num_seqs, "block_size": batch.block_size,
                 "head_dim": batch.head_dim, "num_q_heads": batch.num_q_heads, "num_kv_heads": batch.num_kv_heads,
                 "partition": partition, "fused_append": fused,
+                "shared_prefix": list(step.shared_prefix) if cascade else None,
                 "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
                 "kv_bytes_logical_per_rank": acct["kv_logical"], "kv_bytes_unique_per_rank": acct["kv_unique"],
                 "parallelism": f"dp{world} (independent batches per GPU)",

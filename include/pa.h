@@ -205,6 +205,34 @@ PA_API int pa_decode_splitkv(float* part_o, float* part_m, float* part_l, const 
                              pa_dtype dtype, void* stream);
 
 /*
+ * pa_decode_shared_prefix - decode for a batch whose first `group_size`
+ * sequences share their first `prefix_len` tokens through the same physical
+ * blocks (a common prompt: [FP] PagedAttention step 4 and its block-table
+ * example; [PR], RadixAttention's reuse of a prefix's KV state).
+ *
+ * Same output as pa_decode (plus, when k_new/v_new are given, the cache write
+ * of pa_decode_append), computed as a cascade:
+ *   1) the group's G*group_size query rows of each KV head attend to the shared
+ *      prefix pages once, as a dense tile on the tensor cores (read through
+ *      block_tables row 0), giving split-KV partials in slot 0;
+ *   2) every sequence's remaining tokens, in prefix_len-token partitions
+ *      (pa_decode_splitkv with partition_size = prefix_len; partition 0 of the
+ *      group is skipped), the newest token's row written first if given;
+ *   3) pa_merge.
+ * part_o/part_m/part_l: caller workspace [N, Hq, num_partitions(, D)] fp32,
+ * num_partitions >= ceil(max L / prefix_len). Needs prefix_len a positive
+ * multiple of 16 and of B, every group member with L_b > prefix_len, f16 or
+ * bf16. The kernels do not check that the prefix blocks are really shared.
+ */
+PA_API int pa_decode_shared_prefix(void* out, const void* q, const void* k_new, const void* v_new,
+                                   void* k_cache, void* v_cache, const int32_t* block_tables,
+                                   int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                                   int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                   int num_blocks, int prefix_len, int group_size, float* part_o,
+                                   float* part_m, float* part_l, int num_partitions, float scale,
+                                   pa_dtype dtype, void* stream);
+
+/*
  * pa_merge - combine split-KV partitions into the attention output.
  *
  * Log-sum-exp rule over the partitions p < ceil(L_b / S) with part_l > 0

@@ -17,6 +17,22 @@ namespace pa {
 // Device error word of the current device (lives in pa_api.cu).
 unsigned int* device_error_word();
 
+// Shared-prefix mode of the tensor-core prefill kernel: the group's decode
+// queries attend to keys [0, prefix_len) of block-table row 0 and the result
+// lands as split-KV partials in slot 0 of [N, Hq, num_partitions, D].
+struct PrefixPartials {
+  int prefix_len;
+  float* part_o;
+  float* part_m;
+  float* part_l;
+  int num_partitions;
+};
+
+int prefill_tcgen05(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                    int max_blocks_per_seq, const int32_t* context_lens, int num_seqs, int chunk_len,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                    pa_dtype dtype, cudaStream_t stream, const PrefixPartials* pp);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline bool supported_block(int b) { return b == 8 || b == 16 || b == 32 || b == 64 || b == 128; }

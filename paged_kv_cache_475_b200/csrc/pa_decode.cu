@@ -76,6 +76,7 @@ struct DecodeParams {
   float q_scale;             // scale * log2(e)
   const void* k_new;         // fused append: [N, Hkv, D] rows of each sequence's newest token, or null
   const void* v_new;
+  int skip_part0_seqs;       // split mode: partition 0 of sequences below this is computed elsewhere
 };
 
 // Sequence whose context is the r-th longest (ties by index). CTAs are
@@ -211,6 +212,12 @@ decode_kernel(const DecodeParams p) {
   const int part = blockIdx.x;
   const int kvh = blockIdx.y;
   const bool split = p.partition > 0;
+  // A shared prefix's partition was computed once for its whole group; a
+  // group member must reach past the prefix (its newest token is its own).
+  if (split && part == 0 && static_cast<int>(blockIdx.z) < p.skip_part0_seqs) {
+    if (threadIdx.x == 0 && kvh == 0 && p.context_lens[blockIdx.z] <= p.partition) set_error(p.err, PA_DEVERR_CONTEXT);
+    return;
+  }
   const int b = p.longest_first
                     ? longest_first_seq(p.context_lens, p.num_seqs, blockIdx.z,
                                         reinterpret_cast<int*>(smem + M::kValidOff + NW * STAGES * 4))
@@ -842,6 +849,8 @@ extern "C" PA_API int pa_decode_splitkv(float* part_o, float* part_m, float* par
 }
 
 namespace pa {
+int launch_merge_any(void* out, const float* po, const float* pm, const float* pl, const int32_t* lens, int rows,
+                     int Hq, int D, int partition, int np, pa_dtype dt, cudaStream_t s);
 template <typename T>
 int launch_merge(void* out, const float* po, const float* pm, const float* pl, const int32_t* lens, int rows,
                  int Hq, int D, int partition, int np, cudaStream_t s) {
@@ -877,6 +886,73 @@ extern "C" PA_API int pa_merge(void* out, const float* part_o, const float* part
                                                      num_q_heads, head_dim, partition_size, num_partitions, s);
   }
   return PA_ERR_DTYPE;
+}
+
+namespace pa {
+int launch_merge_any(void* out, const float* po, const float* pm, const float* pl, const int32_t* lens, int rows,
+                     int Hq, int D, int partition, int np, pa_dtype dt, cudaStream_t s) {
+  switch (dt) {
+    case PA_F32: return launch_merge<float>(out, po, pm, pl, lens, rows, Hq, D, partition, np, s);
+    case PA_F16: return launch_merge<__half>(out, po, pm, pl, lens, rows, Hq, D, partition, np, s);
+    case PA_BF16: return launch_merge<__nv_bfloat16>(out, po, pm, pl, lens, rows, Hq, D, partition, np, s);
+  }
+  return PA_ERR_DTYPE;
+}
+}  // namespace pa
+
+extern "C" PA_API int pa_decode_shared_prefix(void* out, const void* q, const void* k_new, const void* v_new,
+                                              void* k_cache, void* v_cache, const int32_t* block_tables,
+                                              int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                                              int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                              int num_blocks, int prefix_len, int group_size, float* part_o,
+                                              float* part_m, float* part_l, int num_partitions, float scale,
+                                              pa_dtype dtype, void* stream) {
+  int st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                             num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, dtype);
+  if (st != PA_OK || num_seqs == 0) return st;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_DTYPE;
+  if (!out || !part_o || !part_m || !part_l) return PA_ERR_NULL;
+  if ((k_new == nullptr) != (v_new == nullptr)) return PA_ERR_NULL;
+  if ((k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new)) || !aligned16(part_o)) return PA_ERR_ALIGN;
+  if (prefix_len <= 0 || prefix_len % kTile || prefix_len % block_size || group_size < 0 || group_size > num_seqs)
+    return PA_ERR_SHAPE;
+  if (num_partitions <= 0) return PA_ERR_WORKSPACE;
+  if (num_seqs > 65535 || num_partitions > (1 << 30)) return PA_ERR_SHAPE;
+  cudaStream_t s = (cudaStream_t)stream;
+  // 1) the shared prefix, once for the whole group, on the tensor cores -> slot 0
+  if (group_size > 0) {
+    PrefixPartials pp{prefix_len, part_o, part_m, part_l, num_partitions};
+    st = prefill_tcgen05(nullptr, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, 1, group_size,
+                         num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, dtype, s, &pp);
+    if (st != PA_OK) return st;
+  }
+  // 2) every sequence's own tokens in prefix_len-token partitions (partition 0
+  //    of the group comes from step 1), with the newest token's K/V written
+  DecodeParams prm{};
+  prm.part_o = part_o;
+  prm.part_m = part_m;
+  prm.part_l = part_l;
+  prm.q = q;
+  prm.k_cache = k_cache;
+  prm.v_cache = v_cache;
+  prm.k_new = k_new;
+  prm.v_new = v_new;
+  prm.block_tables = block_tables;
+  prm.context_lens = context_lens;
+  prm.max_blocks = max_blocks_per_seq;
+  prm.num_seqs = num_seqs;
+  prm.num_q_heads = num_q_heads;
+  prm.num_kv_heads = num_kv_heads;
+  prm.block_size = block_size;
+  prm.num_blocks = num_blocks;
+  prm.partition = prefix_len;
+  prm.num_parts = num_partitions;
+  prm.skip_part0_seqs = group_size;
+  st = run_decode(prm, head_dim, scale, dtype, num_partitions, s);
+  if (st != PA_OK) return st;
+  // 3) log-sum-exp merge of all partitions
+  return launch_merge_any(out, part_o, part_m, part_l, context_lens, num_seqs * num_q_heads, num_q_heads, head_dim,
+                          prefix_len, num_partitions, dtype, s);
 }
 
 // ---------------------------------------------------------------------------

@@ -67,6 +67,15 @@ struct Params {
   int chunk_rows;      // rows per TMA box = min(B, 16)
   int oob_row;         // a row coordinate past the pool: TMA reads zeros there
   float scale_log2;
+  // Shared-prefix mode (prefix_len > 0): the "chunk" is a group of decode
+  // queries (one per sequence) that all see keys [0, prefix_len) of block
+  // table row 0, without a causal mask; the result is written as split-KV
+  // partials (slot 0 of [N, Hq, part_np, D]) instead of normalised rows.
+  int prefix_len;
+  float* part_o;
+  float* part_m;
+  float* part_l;
+  int part_np;
 };
 
 template <int D>
@@ -328,15 +337,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const int qt = gridDim.x - 1 - blockIdx.x;  // latest (heaviest) query tiles first
   const int kvh = blockIdx.y, b = blockIdx.z;
   const int C = p.chunk, B = p.block_size;
-  int L = p.context_lens[b];
+  const bool prefix_mode = p.prefix_len > 0;
+  int L = prefix_mode ? p.prefix_len : p.context_lens[b];
   if (L < 0 || L > p.max_blocks * B) {
     if (threadIdx.x == 0) set_error(p.err, PA_DEVERR_CONTEXT);
     L = L < 0 ? 0 : p.max_blocks * B;
   }
   const int i0 = qt * QT;
   const int q_hi = min(C, i0 + QT);
-  const int pos_lo = L - C + i0;
-  const int pos_hi = L - C + q_hi - 1;
+  // causal: query i at position L - C + i; prefix mode: every query sees all L keys
+  const int pos_lo = prefix_mode ? L - 1 : L - C + i0;
+  const int pos_hi = prefix_mode ? L - 1 : L - C + q_hi - 1;
   const int n_keys = pos_hi + 1 > 0 ? pos_hi + 1 : 0;
   const int n_tiles = (n_keys + kN - 1) / kN;
 
@@ -508,7 +519,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int quad = warp & 3, half = warp >> 2;
     const int r = quad * 32 + lane;            // row = TMEM lane
     const int i = i0 + r / G, g = r % G;
-    const int pos = L - C + i;
+    const int pos = prefix_mode ? L - 1 : L - C + i;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const int bar_id = 1 + quad;
     float* red = reinterpret_cast<float*>(smem + S::oRed);
@@ -629,6 +640,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const bool store = i < C;
       T* orow = static_cast<T*>(p.out) +
                 ((static_cast<int64_t>(b) * C + (store ? i : 0)) * p.num_q_heads + kvh * G + g) * D + half * HD;
+      // prefix mode: partial state of row (sequence i, head kvh*G + g), slot 0
+      const int64_t prow = (static_cast<int64_t>(store ? i : 0) * p.num_q_heads + kvh * G + g) * p.part_np;
+      if (prefix_mode && store && half == 0) {
+        p.part_m[prow] = (den > 0.f && n_tiles > 0) ? Ms * 0.6931471805599453f : -INFINITY;
+        p.part_l[prow] = n_tiles > 0 ? den : 0.f;
+      }
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
         float o[32], o1[32];
@@ -641,6 +658,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           for (int e = 0; e < 32; ++e) o[e] = o1[e] = 0.f;
         }
         if (!store) continue;
+        if (prefix_mode) {  // unnormalised: sum_t 2^(s_t - M) v_t
+          float* dst = p.part_o + prow * D + half * HD + c * 32;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + e) = make_float4(o[e] * f0 + o1[e] * f1, o[e + 1] * f0 + o1[e + 1] * f1,
+                                                              o[e + 2] * f0 + o1[e + 2] * f1, o[e + 3] * f0 + o1[e + 3] * f1);
+          continue;
+        }
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = (o[e] * f0 + o1[e] * f1) * inv;
 #pragma unroll
@@ -743,11 +768,11 @@ int by_group(const Params& prm, int G, const void* q, const void* k, const void*
 int prefill_tcgen05(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
                     int max_blocks_per_seq, const int32_t* context_lens, int num_seqs, int chunk_len,
                     int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
-                    pa_dtype dtype, cudaStream_t stream) {
+                    pa_dtype dtype, cudaStream_t stream, const PrefixPartials* pp) {
   const long long pool_rows = static_cast<long long>(num_blocks) * num_kv_heads * block_size;
   if (pool_rows + 16 > 0x7fffffffLL || static_cast<long long>(num_seqs) * chunk_len > 0x7fffffffLL)
     return PA_ERR_SHAPE;
-  if (!aligned16(out) || (reinterpret_cast<uintptr_t>(q) & 15)) return PA_ERR_ALIGN;
+  if ((out && !aligned16(out)) || (reinterpret_cast<uintptr_t>(q) & 15)) return PA_ERR_ALIGN;
   tc::Params prm{};
   prm.out = out;
   prm.block_tables = block_tables;
@@ -763,6 +788,13 @@ int prefill_tcgen05(void* out, const void* q, const void* k_cache, const void* v
   prm.chunk_rows = block_size < 16 ? block_size : 16;
   prm.oob_row = static_cast<int>(pool_rows);  // first row past the pool: TMA reads zeros
   prm.scale_log2 = scale * tc::kLog2e;
+  if (pp) {
+    prm.prefix_len = pp->prefix_len;
+    prm.part_o = pp->part_o;
+    prm.part_m = pp->part_m;
+    prm.part_l = pp->part_l;
+    prm.part_np = pp->num_partitions;
+  }
   const int G = num_q_heads / num_kv_heads;
   if (dtype == PA_BF16) {
     if (head_dim == 128) return tc::by_group<__nv_bfloat16, 128>(prm, G, q, k_cache, v_cache, pool_rows, stream);
@@ -797,5 +829,5 @@ extern "C" PA_API int pa_prefill_chunk(void* out, const void* q, const void* k_c
   if (num_seqs > 65535 || num_kv_heads > 65535) return PA_ERR_SHAPE;
   return prefill_tcgen05(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
                          chunk_len, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, dtype,
-                         (cudaStream_t)stream);
+                         (cudaStream_t)stream, nullptr);
 }

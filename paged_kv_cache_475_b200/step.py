@@ -11,8 +11,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (pa_decode, pa_decode_append, pa_decode_splitkv, pa_merge, pa_prefill_chunk,
-               pa_reshape_and_cache, pa_slot_mapping, pa_splitkv_num_partitions)
+from . import (pa_decode, pa_decode_append, pa_decode_shared_prefix, pa_decode_splitkv, pa_merge,
+               pa_prefill_chunk, pa_reshape_and_cache, pa_slot_mapping, pa_splitkv_num_partitions)
 
 NUM_SMS_B200 = 148
 
@@ -39,12 +39,33 @@ class DecodeStep:
     of k_new/v_new is sequence b's newest, at position context_lens[b] - 1),
     the append is folded into the decode kernel (pa_decode_append: one launch).
     "auto" picks it whenever those conditions hold by construction.
+
+    shared_prefix=(prefix_len, group_size): sequences 0..group_size-1 share the
+    blocks of their first prefix_len tokens; the step then runs the cascade of
+    pa_decode_shared_prefix (prefix once per group on the tensor cores, the
+    rest split-KV, merge), with the newest tokens' K/V written on the way.
     """
 
     def __init__(self, num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
                  max_context_len: int, dtype: torch.dtype, num_new_tokens: int | None = None,
-                 partition: int | None | str = "auto", fused_append: bool | str = "auto", device="cuda"):
+                 partition: int | None | str = "auto", fused_append: bool | str = "auto",
+                 shared_prefix: tuple[int, int] | None = None, device="cuda"):
         self.N, self.Hq, self.D = num_seqs, num_q_heads, head_dim
+        self.shared_prefix = shared_prefix
+        if shared_prefix is not None:
+            prefix_len, _ = shared_prefix
+            self.num_parts = pa_splitkv_num_partitions(max_context_len, prefix_len)
+            self.part_o = torch.empty((num_seqs, num_q_heads, self.num_parts, head_dim), dtype=torch.float32,
+                                      device=device)
+            self.part_m = torch.empty((num_seqs, num_q_heads, self.num_parts), dtype=torch.float32, device=device)
+            self.part_l = torch.empty_like(self.part_m)
+            self.out = torch.empty((num_seqs, num_q_heads, head_dim), dtype=dtype, device=device)
+            self.fused = num_new_tokens is None or num_new_tokens == num_seqs
+            self.partition = prefix_len
+            self.launches_per_call = 3 if self.fused else 5
+            self.slot_mapping = torch.empty(num_seqs if num_new_tokens is None else num_new_tokens,
+                                            dtype=torch.int64, device=device)
+            return
         if partition == "auto":
             partition = choose_partition(num_seqs, num_kv_heads, max_context_len)
         self.partition = partition
@@ -65,6 +86,16 @@ class DecodeStep:
 
     def __call__(self, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, new_seq, new_pos,
                  scale: float, stream=None):
+        if self.shared_prefix is not None:
+            prefix_len, group = self.shared_prefix
+            if not self.fused:
+                B = k_cache.shape[2]
+                pa_slot_mapping(self.slot_mapping, block_tables, new_seq, new_pos, B, stream)
+                pa_reshape_and_cache(k_new, v_new, k_cache, v_cache, self.slot_mapping, stream)
+            pa_decode_shared_prefix(self.out, q, k_new if self.fused else None, v_new if self.fused else None,
+                                    k_cache, v_cache, block_tables, context_lens, prefix_len, group,
+                                    self.part_o, self.part_m, self.part_l, scale, stream)
+            return self.out
         if self.fused:
             pa_decode_append(self.out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, scale, stream)
             return self.out
@@ -99,12 +130,20 @@ class PrefillStep:
         return self.out
 
 
-def run_batch(batch, partition: int | None | str = "auto", fused_append: bool | str = "auto"):
-    """Run one step of a workloads.PagedBatch that lives on the GPU; returns the output tensor."""
+def run_batch(batch, partition: int | None | str = "auto", fused_append: bool | str = "auto",
+              shared_prefix: tuple[int, int] | None | str = None):
+    """Run one step of a workloads.PagedBatch that lives on the GPU; returns the output tensor.
+
+    shared_prefix="batch" takes (prefix tokens, group) from the batch's own generator settings.
+    """
+    if shared_prefix == "batch":
+        sp, sg = batch.info.get("shared_prefix_tokens", 0), batch.info.get("shared_group", 0)
+        shared_prefix = (sp, sg) if sp and sg else None
     if batch.chunk == 1:
         step = DecodeStep(batch.num_seqs, batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
                           int(batch.context_lens.max().item()) if batch.num_seqs else 1, batch.q.dtype,
-                          num_new_tokens=batch.new_seq.shape[0], partition=partition, fused_append=fused_append)
+                          num_new_tokens=batch.new_seq.shape[0], partition=partition, fused_append=fused_append,
+                          shared_prefix=shared_prefix)
     else:
         step = PrefillStep(batch.num_seqs, batch.chunk, batch.num_q_heads, batch.head_dim, batch.q.dtype,
                            num_new_tokens=batch.new_seq.shape[0])

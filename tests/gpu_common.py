@@ -19,14 +19,14 @@ def require_gpu():
         pytest.fail("this test needs a CUDA GPU (run with -m 'not gpu' on a CPU-only machine)")
 
 
-def run_gpu(batch_cpu, partition="auto", fused_append="auto"):
+def run_gpu(batch_cpu, partition="auto", fused_append="auto", shared_prefix=None):
     """One step of the batch on the GPU through the C ABI; returns (out, gpu_batch, error_flags)."""
     import paged_kv_cache_475_b200 as pa
     from paged_kv_cache_475_b200.step import run_batch
 
     pa.pa_read_error_flags(clear=True)
     g = batch_cpu.to("cuda")
-    out = run_batch(g, partition, fused_append)
+    out = run_batch(g, partition, fused_append, shared_prefix)
     torch.cuda.synchronize()
     flags = pa.pa_read_error_flags(clear=True)
     return out.cpu(), g, flags

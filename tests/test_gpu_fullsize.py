@@ -53,6 +53,9 @@ def test_chat_trace_full(B):
     out, _, flags = run_gpu(b, partition="auto")
     assert flags == 0
     assert_close(out, ref, "f16", f"chat trace B={B}")
+    out, _, flags = run_gpu(b, shared_prefix="batch")   # the cascade bench.py times
+    assert flags == 0
+    assert_close(out, ref, "f16", f"chat trace shared-prefix B={B}")
 
 
 def test_prefill_chunk_sampled():

@@ -382,3 +382,28 @@ def test_copy_on_write_through_the_block_manager():
     assert torch.equal(gk.cpu().view(torch.int16), okc.view(torch.int16))
     assert_close(out.cpu(), ref, "f16", "copy on write")
     assert pa.pa_read_error_flags() == 0
+
+
+# ---------------------------------------------------------------------------
+# Shared-prefix (cascade) decode
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("B,prefix,G", [(16, 64, 4), (8, 128, 2), (32, 32, 8), (128, 128, 4)])
+def test_decode_shared_prefix(dtype, B, prefix, G):
+    lens = (prefix + 1, prefix + 40, prefix + 300, 17, prefix + 700, 90)
+    b = small_batch(seed=400 + B + prefix, dtype=dtype, B=B, G=G, lens=lens, shared_prefix_tokens=prefix,
+                    shared_group=3)
+    ref, kc, vc, _ = oracle.step(b)
+    for fused in (True, False):
+        out, g, flags = run_gpu(b, fused_append=fused, shared_prefix="batch")
+        assert flags == 0
+        assert_close(out, ref, dtype, f"shared prefix {dtype} B={B} prefix={prefix} fused={fused}")
+        assert torch.equal(g.k_cache.cpu().view(torch.int16), kc.view(torch.int16))
+
+
+def test_decode_shared_prefix_rejects_a_member_inside_the_prefix():
+    import paged_kv_cache_475_b200 as pa
+    b = small_batch(seed=410, lens=(64, 100, 300), shared_prefix_tokens=64, shared_group=2)
+    out, _, flags = run_gpu(b, shared_prefix="batch")   # sequence 0 ends exactly at the prefix end
+    assert flags & pa.DEVERR_CONTEXT
