@@ -214,15 +214,19 @@ PA_API int pa_decode_splitkv(float* part_o, float* part_m, float* part_l, const 
  * of pa_decode_append), computed as a cascade:
  *   1) the group's G*group_size query rows of each KV head attend to the shared
  *      prefix pages once, as a dense tile on the tensor cores (read through
- *      block_tables row 0), giving split-KV partials in slot 0;
- *   2) every sequence's remaining tokens, in prefix_len-token partitions
- *      (pa_decode_splitkv with partition_size = prefix_len; partition 0 of the
- *      group is skipped), the newest token's row written first if given;
- *   3) pa_merge.
+ *      block_tables row 0); the prefix keys are cut into S = 4, 2 or 1 equal
+ *      ranges (multiples of 128 keys, S + 1 <= num_partitions), one partial
+ *      slot each;
+ *   2) one pass per (sequence, KV head) over the sequence's own tokens: group
+ *      members from token prefix_len on, written as partials into slot S; all
+ *      other sequences whole, written straight to `out`; the newest token's
+ *      row written first if given;
+ *   3) the group's rows: log-sum-exp merge of slots 0..S.
  * part_o/part_m/part_l: caller workspace [N, Hq, num_partitions(, D)] fp32,
- * num_partitions >= ceil(max L / prefix_len). Needs prefix_len a positive
- * multiple of 16 and of B, every group member with L_b > prefix_len, f16 or
- * bf16. The kernels do not check that the prefix blocks are really shared.
+ * num_partitions >= 2 (5 lets S reach 4). Needs prefix_len a positive
+ * multiple of 16 and of B, every group member with L_b > prefix_len (else
+ * PA_DEVERR_CONTEXT), f16 or bf16. The kernels do not check that the prefix
+ * blocks are really shared.
  */
 PA_API int pa_decode_shared_prefix(void* out, const void* q, const void* k_new, const void* v_new,
                                    void* k_cache, void* v_cache, const int32_t* block_tables,

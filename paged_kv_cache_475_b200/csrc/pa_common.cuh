@@ -18,14 +18,16 @@ namespace pa {
 unsigned int* device_error_word();
 
 // Shared-prefix mode of the tensor-core prefill kernel: the group's decode
-// queries attend to keys [0, prefix_len) of block-table row 0 and the result
-// lands as split-KV partials in slot 0 of [N, Hq, num_partitions, D].
+// queries attend to keys [0, prefix_len) of block-table row 0, cut into
+// key_splits ranges, and the results land as split-KV partials in slots
+// 0..key_splits-1 of [N, Hq, num_partitions, D].
 struct PrefixPartials {
   int prefix_len;
   float* part_o;
   float* part_m;
   float* part_l;
   int num_partitions;
+  int key_splits;  // the prefix keys are cut into this many equal ranges, one partial slot each
 };
 
 int prefill_tcgen05(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,

@@ -77,20 +77,28 @@ struct DecodeParams {
   const void* k_new;         // fused append: [N, Hkv, D] rows of each sequence's newest token, or null
   const void* v_new;
   int skip_part0_seqs;       // split mode: partition 0 of sequences below this is computed elsewhere
+  // Shared-prefix cascade (single pass, cascade_prefix > 0): sequences below
+  // cascade_group start at token cascade_prefix and write partials into slot
+  // cascade_slot of [N, Hq, num_parts, D]; the others write their rows to out.
+  int cascade_prefix;
+  int cascade_group;
+  int cascade_slot;
 };
 
 // Sequence whose context is the r-th longest (ties by index). CTAs are
 // dispatched in z order, so the longest contexts start first and short ones
 // fill the tail (greedy longest-processing-time scheduling). O(N^2 / threads)
 // compares per CTA, used for small batches only.
-__device__ inline int longest_first_seq(const int32_t* lens, int n, int r, int* slot) {
+// Work of sequence j is its length minus `skip` tokens when j < group.
+__device__ inline int longest_first_seq(const int32_t* lens, int n, int r, int* slot, int group = 0,
+                                        int skip = 0) {
   if (threadIdx.x == 0) *slot = r;
   __syncthreads();
   for (int j = threadIdx.x; j < n; j += blockDim.x) {
-    const int Lj = lens[j];
+    const int Lj = lens[j] - (j < group ? skip : 0);
     int rank = 0;
     for (int i = 0; i < n; ++i) {
-      const int Li = lens[i];
+      const int Li = lens[i] - (i < group ? skip : 0);
       rank += (Li > Lj) || (Li == Lj && i < j);
     }
     if (rank == r) *slot = j;
@@ -220,8 +228,12 @@ decode_kernel(const DecodeParams p) {
   }
   const int b = p.longest_first
                     ? longest_first_seq(p.context_lens, p.num_seqs, blockIdx.z,
-                                        reinterpret_cast<int*>(smem + M::kValidOff + NW * STAGES * 4))
+                                        reinterpret_cast<int*>(smem + M::kValidOff + NW * STAGES * 4),
+                                        p.cascade_group, p.cascade_prefix)
                     : static_cast<int>(blockIdx.z);
+  const bool cascade_member = p.cascade_prefix > 0 && b < p.cascade_group;
+  if (cascade_member && threadIdx.x == 0 && kvh == 0 && p.context_lens[b] <= p.cascade_prefix)
+    set_error(p.err, PA_DEVERR_CONTEXT);
 
   // ---- context range of this CTA -------------------------------------------
   int L = p.context_lens[b];
@@ -231,7 +243,7 @@ decode_kernel(const DecodeParams p) {
   }
   if (split && part == p.num_parts - 1 && L > p.num_parts * p.partition && threadIdx.x == 0)
     set_error(p.err, PA_DEVERR_CONTEXT);
-  const int t_begin = split ? part * p.partition : 0;
+  const int t_begin = split ? part * p.partition : (cascade_member ? p.cascade_prefix : 0);
   int t_end = split ? min(L, t_begin + p.partition) : L;
   if (t_end < t_begin) t_end = t_begin;
   const int n_tiles = (t_end - t_begin + kTile - 1) / kTile;
@@ -569,8 +581,9 @@ decode_kernel(const DecodeParams p) {
       }
     }
     const int h = kvh * G + g;
-    if (split) {
-      const int64_t row = (static_cast<int64_t>(b) * p.num_q_heads + h) * p.num_parts + part;
+    if (split || cascade_member) {
+      const int slot = split ? part : p.cascade_slot;
+      const int64_t row = (static_cast<int64_t>(b) * p.num_q_heads + h) * p.num_parts + slot;
       p.part_o[row * D + d] = o;
       if (d == 0) {
         p.part_m[row] = Mx == -INFINITY ? -INFINITY : Mx * kLn2;
@@ -618,10 +631,14 @@ merge_kernel(T* __restrict__ out, const float* __restrict__ part_o, const float*
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int row = blockIdx.x;  // b * Hq + h
   const int b = row / num_q_heads;
-  int L = context_lens[b];
-  L = L < 0 ? 0 : L;
-  int np = (L + partition - 1) / partition;
-  np = np > num_parts ? num_parts : np;
+  // partition < 0 (cascade): the first -partition slots of each row are live
+  int np = partition < 0 ? (-partition < num_parts ? -partition : num_parts) : num_parts;
+  if (partition > 0) {
+    int L = context_lens[b];
+    L = L < 0 ? 0 : L;
+    np = (L + partition - 1) / partition;
+    np = np > num_parts ? num_parts : np;
+  }
   const float* po = part_o + static_cast<int64_t>(row) * num_parts * D;
   const float* pm = part_m + static_cast<int64_t>(row) * num_parts;
   const float* pl = part_l + static_cast<int64_t>(row) * num_parts;
@@ -851,10 +868,9 @@ extern "C" PA_API int pa_decode_splitkv(float* part_o, float* part_m, float* par
 namespace pa {
 int launch_merge_any(void* out, const float* po, const float* pm, const float* pl, const int32_t* lens, int rows,
                      int Hq, int D, int partition, int np, pa_dtype dt, cudaStream_t s);
-template <typename T>
-int launch_merge(void* out, const float* po, const float* pm, const float* pl, const int32_t* lens, int rows,
-                 int Hq, int D, int partition, int np, cudaStream_t s) {
-  constexpr int MW = 8;
+template <typename T, int MW>
+int launch_merge_mw(void* out, const float* po, const float* pm, const float* pl, const int32_t* lens, int rows,
+                    int Hq, int D, int partition, int np, cudaStream_t s) {
   if (D == 64)
     merge_kernel<T, 64, MW><<<rows, MW * 32, 0, s>>>(static_cast<T*>(out), po, pm, pl, lens, Hq, partition, np);
   else if (D == 128)
@@ -862,6 +878,14 @@ int launch_merge(void* out, const float* po, const float* pm, const float* pl, c
   else
     return PA_ERR_UNSUPPORTED;
   return launch_status();
+}
+// 8 warps per row when there are many partitions, 2 when there are few.
+template <typename T>
+int launch_merge(void* out, const float* po, const float* pm, const float* pl, const int32_t* lens, int rows,
+                 int Hq, int D, int partition, int np, cudaStream_t s) {
+  const int live = partition < 0 ? -partition : np;
+  if (live <= 8) return launch_merge_mw<T, 2>(out, po, pm, pl, lens, rows, Hq, D, partition, np, s);
+  return launch_merge_mw<T, 8>(out, po, pm, pl, lens, rows, Hq, D, partition, np, s);
 }
 }  // namespace pa
 
@@ -916,19 +940,27 @@ extern "C" PA_API int pa_decode_shared_prefix(void* out, const void* q, const vo
   if ((k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new)) || !aligned16(part_o)) return PA_ERR_ALIGN;
   if (prefix_len <= 0 || prefix_len % kTile || prefix_len % block_size || group_size < 0 || group_size > num_seqs)
     return PA_ERR_SHAPE;
-  if (num_partitions <= 0) return PA_ERR_WORKSPACE;
-  if (num_seqs > 65535 || num_partitions > (1 << 30)) return PA_ERR_SHAPE;
+  if (num_partitions < 2) return PA_ERR_WORKSPACE;
+  if (num_seqs > 65535) return PA_ERR_SHAPE;
   cudaStream_t s = (cudaStream_t)stream;
-  // 1) the shared prefix, once for the whole group, on the tensor cores -> slot 0
+  // Split the prefix keys over up to 4 CTA rows (each a multiple of 128 keys)
+  // so the prefix pass fills the GPU; its slots are 0..splits-1, the
+  // suffix pass writes slot `splits`.
+  int splits = 1;
+  for (int c : {4, 2})
+    if (splits == 1 && prefix_len % (128 * c) == 0 && c + 1 <= num_partitions) splits = c;
+  // 1) the shared prefix, once for the whole group, on the tensor cores
   if (group_size > 0) {
-    PrefixPartials pp{prefix_len, part_o, part_m, part_l, num_partitions};
+    PrefixPartials pp{prefix_len, part_o, part_m, part_l, num_partitions, splits};
     st = prefill_tcgen05(nullptr, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, 1, group_size,
                          num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, dtype, s, &pp);
     if (st != PA_OK) return st;
   }
-  // 2) every sequence's own tokens in prefix_len-token partitions (partition 0
-  //    of the group comes from step 1), with the newest token's K/V written
+  // 2) every sequence's own tokens in one pass per (sequence, KV head): group
+  //    members from prefix_len on (partials), the others whole (final rows);
+  //    the newest token's K/V written on the way when given
   DecodeParams prm{};
+  prm.out = out;
   prm.part_o = part_o;
   prm.part_m = part_m;
   prm.part_l = part_l;
@@ -945,14 +977,17 @@ extern "C" PA_API int pa_decode_shared_prefix(void* out, const void* q, const vo
   prm.num_kv_heads = num_kv_heads;
   prm.block_size = block_size;
   prm.num_blocks = num_blocks;
-  prm.partition = prefix_len;
+  prm.partition = 0;
   prm.num_parts = num_partitions;
-  prm.skip_part0_seqs = group_size;
-  st = run_decode(prm, head_dim, scale, dtype, num_partitions, s);
-  if (st != PA_OK) return st;
-  // 3) log-sum-exp merge of all partitions
-  return launch_merge_any(out, part_o, part_m, part_l, context_lens, num_seqs * num_q_heads, num_q_heads, head_dim,
-                          prefix_len, num_partitions, dtype, s);
+  prm.cascade_prefix = prefix_len;
+  prm.cascade_group = group_size;
+  prm.cascade_slot = splits;
+  prm.longest_first = num_seqs > 1 && num_seqs <= PA_DECODE_LPT_MAX_SEQS;
+  st = run_decode(prm, head_dim, scale, dtype, 1, s);
+  if (st != PA_OK || group_size == 0) return st;
+  // 3) the group's rows: log-sum-exp merge of the prefix slots and the suffix slot
+  return launch_merge_any(out, part_o, part_m, part_l, context_lens, group_size * num_q_heads, num_q_heads,
+                          head_dim, -(splits + 1), num_partitions, dtype, s);
 }
 
 // ---------------------------------------------------------------------------

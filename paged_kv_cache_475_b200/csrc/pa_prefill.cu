@@ -76,6 +76,7 @@ struct Params {
   float* part_m;
   float* part_l;
   int part_np;
+  int key_splits;
 };
 
 template <int D>
@@ -335,20 +336,24 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = gridDim.x - 1 - blockIdx.x;  // latest (heaviest) query tiles first
-  const int kvh = blockIdx.y, b = blockIdx.z;
-  const int C = p.chunk, B = p.block_size;
   const bool prefix_mode = p.prefix_len > 0;
-  int L = prefix_mode ? p.prefix_len : p.context_lens[b];
+  // prefix mode: z selects one of key_splits equal key ranges [key0, key0 + per)
+  const int kvh = blockIdx.y, b = prefix_mode ? 0 : static_cast<int>(blockIdx.z);
+  const int split = prefix_mode ? static_cast<int>(blockIdx.z) : 0;
+  const int C = p.chunk, B = p.block_size;
+  const int per = prefix_mode ? p.prefix_len / p.key_splits : 0;
+  const int key0 = split * per;                 // first key of this CTA's range (0 when causal)
+  int L = prefix_mode ? key0 + per : p.context_lens[b];  // keys [key0, L)
   if (L < 0 || L > p.max_blocks * B) {
     if (threadIdx.x == 0) set_error(p.err, PA_DEVERR_CONTEXT);
     L = L < 0 ? 0 : p.max_blocks * B;
   }
   const int i0 = qt * QT;
   const int q_hi = min(C, i0 + QT);
-  // causal: query i at position L - C + i; prefix mode: every query sees all L keys
+  // causal: query i at position L - C + i; prefix mode: every query sees all keys of the range
   const int pos_lo = prefix_mode ? L - 1 : L - C + i0;
   const int pos_hi = prefix_mode ? L - 1 : L - C + q_hi - 1;
-  const int n_keys = pos_hi + 1 > 0 ? pos_hi + 1 : 0;
+  const int n_keys = pos_hi + 1 > key0 ? pos_hi + 1 - key0 : 0;
   const int n_tiles = (n_keys + kN - 1) / kN;
 
   if (threadIdx.x == 0) {
@@ -409,7 +414,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int c = lane + 32 * u;
-          const int t0 = j * kN + c * R;
+          const int t0 = key0 + j * kN + c * R;
           y[u] = p.oob_row;  // chunks past the context read out of range: zeros
           if (c < chunks && j < n_tiles && t0 < L) {
             const int id = bt[t0 / B];
@@ -453,9 +458,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       // V rows past the context inside the last page chunk hold whatever the
       // pool holds there; P is 0 for them but 0 * NaN is NaN, so zero them.
       const int R = p.chunk_rows;
-      const int z0 = L - k * kN;
+      const int z0 = L - (key0 + k * kN);
       if (z0 > 0 && z0 < kN && (L % R) != 0) {
-        const int z1 = min(kN, ((L + R - 1) / R) * R - k * kN);
+        const int z1 = min(kN, ((L + R - 1) / R) * R - (key0 + k * kN));
         const int n16 = (z1 - z0) * KA * 8;  // 16-byte pieces
         for (int e = lane; e < n16; e += 32) {
           const int row = z0 + e / (KA * 8), rest = e % (KA * 8);
@@ -541,7 +546,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tmem_ld32(tS + 32, v + 32);
         tmem_wait_ld();
       }
-      const int t0 = j * kN + half * HC;       // first key of this half
+      const int t0 = key0 + j * kN + half * HC;  // first key of this half
       if (t0 + HC - 1 > pos_lo) {              // causal mask on the diagonal
 #pragma unroll
         for (int e = 0; e < HC; ++e)
@@ -641,7 +646,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       T* orow = static_cast<T*>(p.out) +
                 ((static_cast<int64_t>(b) * C + (store ? i : 0)) * p.num_q_heads + kvh * G + g) * D + half * HD;
       // prefix mode: partial state of row (sequence i, head kvh*G + g), slot 0
-      const int64_t prow = (static_cast<int64_t>(store ? i : 0) * p.num_q_heads + kvh * G + g) * p.part_np;
+      const int64_t prow = (static_cast<int64_t>(store ? i : 0) * p.num_q_heads + kvh * G + g) * p.part_np + split;
       if (prefix_mode && store && half == 0) {
         p.part_m[prow] = (den > 0.f && n_tiles > 0) ? Ms * 0.6931471805599453f : -INFINITY;
         p.part_l[prow] = n_tiles > 0 ? den : 0.f;
@@ -747,7 +752,7 @@ int launch(const Params& prm, const void* q, const void* k_cache, const void* v_
     if (e != cudaSuccess) return record_cuda_error(e, "prefill: set max dynamic shared memory");
     attr_done[dev] = true;
   }
-  dim3 grid((prm.chunk + QT - 1) / QT, prm.num_kv_heads, prm.num_seqs);
+  dim3 grid((prm.chunk + QT - 1) / QT, prm.num_kv_heads, prm.prefix_len > 0 ? prm.key_splits : prm.num_seqs);
   kern<<<grid, kThreads, smem, stream>>>(mq, mk, mv, prm);
   return launch_status();
 }
@@ -794,6 +799,7 @@ int prefill_tcgen05(void* out, const void* q, const void* k_cache, const void* v
     prm.part_m = pp->part_m;
     prm.part_l = pp->part_l;
     prm.part_np = pp->num_partitions;
+    prm.key_splits = pp->key_splits > 0 ? pp->key_splits : 1;
   }
   const int G = num_q_heads / num_kv_heads;
   if (dtype == PA_BF16) {

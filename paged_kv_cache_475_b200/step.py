@@ -54,7 +54,7 @@ class DecodeStep:
         self.shared_prefix = shared_prefix
         if shared_prefix is not None:
             prefix_len, _ = shared_prefix
-            self.num_parts = pa_splitkv_num_partitions(max_context_len, prefix_len)
+            self.num_parts = 5  # up to 4 prefix key ranges + the suffix slot
             self.part_o = torch.empty((num_seqs, num_q_heads, self.num_parts, head_dim), dtype=torch.float32,
                                       device=device)
             self.part_m = torch.empty((num_seqs, num_q_heads, self.num_parts), dtype=torch.float32, device=device)
