@@ -100,3 +100,31 @@ def test_prefill_rejects_f32(lib):
 def test_zero_sized_calls_are_noops(lib):
     assert lib.pa_slot_mapping(None, None, 0, None, None, 0, 0, 16, None) == 0
     assert lib.pa_reshape_and_cache(None, None, None, None, None, 0, 10, 8, 128, 16, 1, None) == 0
+
+
+def _sp_args(**kw):
+    fake = ctypes.c_void_p(16)
+    a = dict(out=fake, q=fake, k_new=None, v_new=None, kc=fake, vc=fake, bt=fake, mb=4, lens=fake, N=4, Hq=8,
+             Hkv=2, D=128, B=16, P=10, prefix=64, group=2, po=fake, pm=fake, pl=fake, np=5,
+             scale=ctypes.c_float(0.1), dt=1, stream=None)
+    a.update(kw)
+    return list(a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(prefix=24), -2), (dict(prefix=0), -2), (dict(B=32, prefix=48), -2), (dict(group=5), -2),
+    (dict(dt=0), -3), (dict(np=1), -5), (dict(k_new=ctypes.c_void_p(16)), -1), (dict(po=None), -1),
+])
+def test_shared_prefix_rejects_bad_args_on_host(lib, kw, code):
+    assert lib.pa_decode_shared_prefix(*_sp_args(**kw)) == code
+
+
+def test_copy_blocks_and_append_reject_bad_args_on_host(lib):
+    fake = ctypes.c_void_p(16)
+    assert lib.pa_copy_blocks(fake, fake, 4, fake, fake, 4, fake, fake, 0, 2, 128, 16, 1, None) == 0  # no pairs
+    assert lib.pa_copy_blocks(None, fake, 4, fake, fake, 4, fake, fake, 1, 2, 128, 16, 1, None) == -1
+    assert lib.pa_copy_blocks(fake, fake, 4, fake, fake, 4, fake, fake, 1, 2, 128, 16, 9, None) == -3
+    args = [fake, fake, None, fake, fake, fake, fake, 4, fake, 2, 8, 2, 128, 16, 10, ctypes.c_float(0.1), 1, None]
+    assert lib.pa_decode_append(*args) == -1                       # k_new missing
+    args[2] = ctypes.c_void_p(24)
+    assert lib.pa_decode_append(*args) == -7                       # k_new misaligned
