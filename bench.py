@@ -130,52 +130,80 @@ def source_hash(files):
 
 
 class ClockSampler:
-    """nvidia-smi samples (every 200 ms) of SM clock and throttle reasons while the bench runs."""
+    """nvidia-smi samples (every 200 ms) of SM clock and throttle reasons around the timed region.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Each sample carries nvidia-smi's own timestamp. stop() keeps the samples
+    that fall inside the timed region (widened by one sampling period on each
+    side, so that a timed region shorter than the period still gets the
+    samples that bracket it) and waits, up to a second, for the first sample
+    after the region so that one always exists.
+    """
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.2
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         self.proc = None
+        self.window = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "-lms", str(int(self.PERIOD_S * 1000))], stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
-        self.t0 = time.time()
+            return
+        deadline = time.time() + 5.0  # the first sample before any timing starts
+        while time.time() < deadline and not self._rows():
+            time.sleep(0.05)
+
+    def _rows(self):
+        import datetime
+
+        rows = []
+        with open(self.f.name) as fh:
+            for line in fh.read().splitlines():
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+                except ValueError:
+                    continue
+        return rows
+
+    def mark(self, t0, t1):
+        """Host wall-clock bounds of the timed region (time.time() before its first launch, after its sync)."""
+        self.window = (t0, t1)
 
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        t0, t1 = self.window if self.window else (0.0, float("inf"))
+        deadline = time.time() + 1.0
+        while time.time() < deadline and not any(r[0] >= t1 for r in self._rows()):
+            time.sleep(0.05)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        self.f.flush()
-        self.f.seek(0)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.f.read().splitlines():
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
+        rows = self._rows()
         os.unlink(self.f.name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+        inside = [r for r in rows if t0 - self.PERIOD_S <= r[0] <= t1 + self.PERIOD_S]
+        if not inside:  # the sample nearest the region
+            inside = sorted(rows, key=lambda r: min(abs(r[0] - t0), abs(r[0] - t1)))[:1]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = {n for r in inside for n, v in zip(names, r[3]) if v.lower() == "active"}
+        sm = [r[1] for r in inside]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max((r[2] for r in inside),
+                                                                                     default=None),
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
@@ -379,6 +407,16 @@ def run_ours(args):
             if ev is not None:
                 ev[1].record(stream)
             return
+        if fused and partition:
+            if ev is not None:
+                ev[0].record(stream)
+            pa.pa_decode_splitkv_append(step.part_o, step.part_m, step.part_l, batch.q, batch.k_new, batch.v_new,
+                                        batch.k_cache, batch.v_cache, batch.block_tables, batch.context_lens,
+                                        partition, batch.scale)
+            if ev is not None:
+                ev[1].record(stream)
+            pa.pa_merge(step.out, step.part_o, step.part_m, step.part_l, batch.context_lens, partition)
+            return
         if fused:
             if ev is not None:
                 ev[0].record(stream)
@@ -417,11 +455,13 @@ def run_ours(args):
     K = args.steps
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0 = time.time()
     t_start.record(stream)
     for i in range(K):
         run_step(evs[i])
     t_end.record(stream)
     torch.cuda.synchronize()
+    sampler.mark(w0, time.time())
     barrier(world)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -450,7 +490,8 @@ def run_ours(args):
         value = sum_over_ranks(units_rank, world) / (ms_step / 1e3) / 1e9
         unit = "GB/s"
         kname = ("pa_decode_shared_prefix" if cascade else
-                 "pa_decode_append" if fused else ("pa_decode_splitkv" if partition else "pa_decode"))
+                 ("pa_decode_splitkv_append" if partition else "pa_decode_append") if fused else
+                 ("pa_decode_splitkv" if partition else "pa_decode"))
         attend_bytes = acct["attend_unique"] + (acct["append"] if fused else 0)
         achieved = attend_bytes / (kern_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",

@@ -237,6 +237,20 @@ PA_API int pa_decode_shared_prefix(void* out, const void* q, const void* k_new, 
                                    pa_dtype dtype, void* stream);
 
 /*
+ * pa_decode_splitkv_append - pa_decode_splitkv with the step's cache write
+ * folded in, like pa_decode_append: the CTA whose partition holds position
+ * context_lens[b] - 1 writes k_new[b] / v_new[b] ([N, Hkv, D]) into that slot
+ * before reading it. Same partials and requirements as pa_decode_splitkv.
+ */
+PA_API int pa_decode_splitkv_append(float* part_o, float* part_m, float* part_l, const void* q,
+                                    const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                                    const int32_t* block_tables, int max_blocks_per_seq,
+                                    const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                    int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                    int partition_size, int num_partitions, float scale, pa_dtype dtype,
+                                    void* stream);
+
+/*
  * pa_merge - combine split-KV partitions into the attention output.
  *
  * Log-sum-exp rule over the partitions p < ceil(L_b / S) with part_l > 0

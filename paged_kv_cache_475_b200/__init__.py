@@ -47,6 +47,8 @@ _SIGS = {
     "pa_splitkv_num_partitions": [_i, _i],
     "pa_decode_splitkv": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                           _i, _vp],
+    "pa_decode_splitkv_append": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                 _i, _f, _i, _vp],
     "pa_merge": [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp],
     "pa_prefill_chunk": [_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp],
     "pa_decode_splitkv_noalloc": [_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
@@ -254,6 +256,27 @@ def pa_decode_shared_prefix(out, q, k_new, v_new, k_cache, v_cache, block_tables
                                         Hkv, D, B, P, int(prefix_len), int(group_size), _ptr(part_o), _ptr(part_m),
                                         _ptr(part_l), NP, float(scale), _dtype_code(q), _stream(stream)),
            "pa_decode_shared_prefix")
+
+
+def pa_decode_splitkv_append(part_o, part_m, part_l, q, k_new, v_new, k_cache, v_cache, block_tables,
+                             context_lens, partition_size: int, scale: float, stream=None):
+    """pa_decode_splitkv plus the write of each sequence's newest K/V row (k_new/v_new [N, Hkv, D])."""
+    _need(q, "q", None, 3)
+    _need(part_o, "part_o", torch.float32, 4)
+    _need(part_m, "part_m", torch.float32, 3)
+    _need(part_l, "part_l", torch.float32, 3)
+    P, Hkv, B, D, N = _cache_dims(q, k_cache, v_cache, block_tables, context_lens)
+    for n, t in (("k_new", k_new), ("v_new", v_new)):
+        _need(t, n, q.dtype, 3)
+        if t.shape != (N, Hkv, D):
+            raise ValueError(f"{n} must be [N, Hkv, D]")
+    NP = part_o.shape[2]
+    if part_o.shape != (N, q.shape[1], NP, D) or part_m.shape != (N, q.shape[1], NP) or part_l.shape != part_m.shape:
+        raise ValueError("partial buffers must be [N, Hq, NP, D] and [N, Hq, NP]")
+    _check(_lib.pa_decode_splitkv_append(_ptr(part_o), _ptr(part_m), _ptr(part_l), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                         _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1],
+                                         _ptr(context_lens), N, q.shape[1], Hkv, D, B, P, int(partition_size), NP,
+                                         float(scale), _dtype_code(q), _stream(stream)), "pa_decode_splitkv_append")
 
 
 def pa_merge(out, part_o, part_m, part_l, context_lens, partition_size: int, stream=None):

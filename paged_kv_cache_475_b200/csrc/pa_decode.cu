@@ -832,6 +832,44 @@ extern "C" PA_API int pa_decode_append(void* out, const void* q, const void* k_n
   return run_decode(prm, head_dim, scale, dtype, 1, (cudaStream_t)stream);
 }
 
+extern "C" PA_API int pa_decode_splitkv_append(float* part_o, float* part_m, float* part_l, const void* q,
+                                               const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                                               const int32_t* block_tables, int max_blocks_per_seq,
+                                               const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                               int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                               int partition_size, int num_partitions, float scale, pa_dtype dtype,
+                                               void* stream) {
+  if (!k_new || !v_new) return PA_ERR_NULL;
+  if (!aligned16(k_new) || !aligned16(v_new)) return PA_ERR_ALIGN;
+  int st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                             num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, dtype);
+  if (st != PA_OK || num_seqs == 0) return st;
+  if (!part_o || !part_m || !part_l) return PA_ERR_NULL;
+  if (!aligned16(part_o)) return PA_ERR_ALIGN;
+  if (partition_size <= 0 || partition_size % kTile || num_partitions <= 0) return PA_ERR_WORKSPACE;
+  if (num_seqs > 65535 || num_partitions > (1 << 30)) return PA_ERR_SHAPE;
+  DecodeParams prm{};
+  prm.part_o = part_o;
+  prm.part_m = part_m;
+  prm.part_l = part_l;
+  prm.q = q;
+  prm.k_cache = k_cache;
+  prm.v_cache = v_cache;
+  prm.k_new = k_new;
+  prm.v_new = v_new;
+  prm.block_tables = block_tables;
+  prm.context_lens = context_lens;
+  prm.max_blocks = max_blocks_per_seq;
+  prm.num_seqs = num_seqs;
+  prm.num_q_heads = num_q_heads;
+  prm.num_kv_heads = num_kv_heads;
+  prm.block_size = block_size;
+  prm.num_blocks = num_blocks;
+  prm.partition = partition_size;
+  prm.num_parts = num_partitions;
+  return run_decode(prm, head_dim, scale, dtype, num_partitions, (cudaStream_t)stream);
+}
+
 extern "C" PA_API int pa_decode_splitkv(float* part_o, float* part_m, float* part_l, const void* q,
                                         const void* k_cache, const void* v_cache, const int32_t* block_tables,
                                         int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
@@ -885,7 +923,8 @@ int launch_merge(void* out, const float* po, const float* pm, const float* pl, c
                  int Hq, int D, int partition, int np, cudaStream_t s) {
   const int live = partition < 0 ? -partition : np;
   if (live <= 8) return launch_merge_mw<T, 2>(out, po, pm, pl, lens, rows, Hq, D, partition, np, s);
-  return launch_merge_mw<T, 8>(out, po, pm, pl, lens, rows, Hq, D, partition, np, s);
+  if (live <= 64) return launch_merge_mw<T, 8>(out, po, pm, pl, lens, rows, Hq, D, partition, np, s);
+  return launch_merge_mw<T, 32>(out, po, pm, pl, lens, rows, Hq, D, partition, np, s);
 }
 }  // namespace pa
 

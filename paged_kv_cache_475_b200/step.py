@@ -11,8 +11,9 @@ from __future__ import annotations
 
 import torch
 
-from . import (pa_decode, pa_decode_append, pa_decode_shared_prefix, pa_decode_splitkv, pa_merge,
-               pa_prefill_chunk, pa_reshape_and_cache, pa_slot_mapping, pa_splitkv_num_partitions)
+from . import (pa_decode, pa_decode_append, pa_decode_shared_prefix, pa_decode_splitkv,
+               pa_decode_splitkv_append, pa_merge, pa_prefill_chunk, pa_reshape_and_cache, pa_slot_mapping,
+               pa_splitkv_num_partitions)
 
 NUM_SMS_B200 = 148
 
@@ -35,10 +36,11 @@ def choose_partition(num_seqs: int, num_kv_heads: int, max_context_len: int,
 class DecodeStep:
     """Append one token per sequence, then decode-attend over the paged cache.
 
-    fused_append: with no split and exactly one new token per sequence (token b
-    of k_new/v_new is sequence b's newest, at position context_lens[b] - 1),
-    the append is folded into the decode kernel (pa_decode_append: one launch).
-    "auto" picks it whenever those conditions hold by construction.
+    fused_append: with exactly one new token per sequence (token b of
+    k_new/v_new is sequence b's newest, at position context_lens[b] - 1), the
+    append is folded into the decode kernel (pa_decode_append, or
+    pa_decode_splitkv_append + pa_merge when split). "auto" picks it whenever
+    that holds by construction.
 
     shared_prefix=(prefix_len, group_size): sequences 0..group_size-1 share the
     blocks of their first prefix_len tokens; the step then runs the cascade of
@@ -70,9 +72,9 @@ class DecodeStep:
             partition = choose_partition(num_seqs, num_kv_heads, max_context_len)
         self.partition = partition
         one_per_seq = num_new_tokens is None or num_new_tokens == num_seqs
-        self.fused = (not partition and one_per_seq) if fused_append == "auto" else bool(fused_append)
-        if self.fused and (partition or not one_per_seq):
-            raise ValueError("the fused append needs the single-pass decode and one new token per sequence")
+        self.fused = one_per_seq if fused_append == "auto" else bool(fused_append)
+        if self.fused and not one_per_seq:
+            raise ValueError("the fused append needs one new token per sequence")
         T = num_seqs if num_new_tokens is None else num_new_tokens
         self.slot_mapping = torch.empty(T, dtype=torch.int64, device=device)
         self.out = torch.empty((num_seqs, num_q_heads, head_dim), dtype=dtype, device=device)
@@ -82,7 +84,7 @@ class DecodeStep:
                                       device=device)
             self.part_m = torch.empty((num_seqs, num_q_heads, self.num_parts), dtype=torch.float32, device=device)
             self.part_l = torch.empty_like(self.part_m)
-        self.launches_per_call = 1 if self.fused else (4 if partition else 3)
+        self.launches_per_call = (2 if partition else 1) if self.fused else (4 if partition else 3)
 
     def __call__(self, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, new_seq, new_pos,
                  scale: float, stream=None):
@@ -95,6 +97,11 @@ class DecodeStep:
             pa_decode_shared_prefix(self.out, q, k_new if self.fused else None, v_new if self.fused else None,
                                     k_cache, v_cache, block_tables, context_lens, prefix_len, group,
                                     self.part_o, self.part_m, self.part_l, scale, stream)
+            return self.out
+        if self.fused and self.partition:
+            pa_decode_splitkv_append(self.part_o, self.part_m, self.part_l, q, k_new, v_new, k_cache, v_cache,
+                                     block_tables, context_lens, self.partition, scale, stream)
+            pa_merge(self.out, self.part_o, self.part_m, self.part_l, context_lens, self.partition, stream)
             return self.out
         if self.fused:
             pa_decode_append(self.out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, scale, stream)

@@ -201,13 +201,19 @@ def test_decode_bad_block_id_sets_flag_without_fault():
 
 @pytest.mark.parametrize("partition", [16, 64, 512, 4096])
 @pytest.mark.parametrize("B", [8, 16, 128])
-def test_splitkv_partials_and_merge(partition, B):
+@pytest.mark.parametrize("fused", [True, False])
+def test_splitkv_partials_and_merge(partition, B, fused):
+    """Split-KV step with the cache write separate (pa_reshape_and_cache) or folded into the
+    partition holding each sequence's newest token (pa_decode_splitkv_append): the cache equals
+    the oracle's append bit for bit, the merged output and the partials match the oracle."""
     import paged_kv_cache_475_b200 as pa
     b = small_batch(seed=91 + partition + B, B=B, lens=(1, 16, 17, 511, 512, 513, 1400))
-    out, g, flags = run_gpu(b, partition=partition)
+    out, g, flags = run_gpu(b, partition=partition, fused_append=fused)
     assert flags == 0
     ref, kc, vc, _ = oracle.step(b)
-    assert_close(out, ref, "f16", f"merged partition={partition} B={B}")
+    assert_close(out, ref, "f16", f"merged partition={partition} B={B} fused={fused}")
+    assert torch.equal(g.k_cache.cpu().view(torch.int16), kc.view(torch.int16))
+    assert torch.equal(g.v_cache.cpu().view(torch.int16), vc.view(torch.int16))
     # the partials themselves
     NP = pa.pa_splitkv_num_partitions(int(b.context_lens.max()), partition)
     po, pm, pl = pa.splitkv_buffers(b.num_seqs, b.num_q_heads, b.head_dim, NP)
