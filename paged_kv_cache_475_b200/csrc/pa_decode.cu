@@ -87,25 +87,29 @@ struct DecodeParams {
 
 // Sequence whose context is the r-th longest (ties by index). CTAs are
 // dispatched in z order, so the longest contexts start first and short ones
-// fill the tail (greedy longest-processing-time scheduling). O(N^2 / threads)
+// fill the tail (greedy longest-processing-time scheduling). The lengths are
+// staged in shared memory (`work`, n ints) with one coalesced load, then each
+// thread ranks its own sequences against them: O(N^2 / threads) shared-memory
 // compares per CTA, used for small batches only.
 // Work of sequence j is its length minus `skip` tokens when j < group.
-__device__ inline int longest_first_seq(const int32_t* lens, int n, int r, int* slot, int group = 0,
-                                        int skip = 0) {
+__device__ inline int longest_first_seq(const int32_t* lens, int n, int r, int* slot, int* work,
+                                        int group = 0, int skip = 0) {
+  for (int j = threadIdx.x; j < n; j += blockDim.x) work[j] = lens[j] - (j < group ? skip : 0);
   if (threadIdx.x == 0) *slot = r;
   __syncthreads();
   for (int j = threadIdx.x; j < n; j += blockDim.x) {
-    const int Lj = lens[j] - (j < group ? skip : 0);
+    const int Lj = work[j];
     int rank = 0;
+#pragma unroll 8
     for (int i = 0; i < n; ++i) {
-      const int Li = lens[i] - (i < group ? skip : 0);
+      const int Li = work[i];
       rank += (Li > Lj) || (Li == Lj && i < j);
     }
     if (rank == r) *slot = j;
   }
   __syncthreads();
   const int b = *slot;
-  __syncthreads();
+  __syncthreads();  // the staging area is the copy ring, which the caller fills next
   return b;
 }
 
@@ -229,7 +233,7 @@ decode_kernel(const DecodeParams p) {
   const int b = p.longest_first
                     ? longest_first_seq(p.context_lens, p.num_seqs, blockIdx.z,
                                         reinterpret_cast<int*>(smem + M::kValidOff + NW * STAGES * 4),
-                                        p.cascade_group, p.cascade_prefix)
+                                        reinterpret_cast<int*>(smem), p.cascade_group, p.cascade_prefix)
                     : static_cast<int>(blockIdx.z);
   const bool cascade_member = p.cascade_prefix > 0 && b < p.cascade_group;
   if (cascade_member && threadIdx.x == 0 && kvh == 0 && p.context_lens[b] <= p.cascade_prefix)
@@ -266,31 +270,6 @@ decode_kernel(const DecodeParams p) {
   const int B = p.block_size;
   const int n_seq_blocks = (L + B - 1) / B;
 
-  // ---- fused append: the CTA whose range holds position L-1 writes the
-  // sequence's newest K/V row (this KV head) into its slot before reading.
-  // Generic stores, then a proxy fence and a CTA barrier, so the bulk copies
-  // issued below (async proxy) see the row.
-  if (p.k_new != nullptr && L > 0 && t_begin <= L - 1 && L - 1 < t_end) {
-    if (warp == 0) {
-      const int pos = L - 1;
-      const int phys = bt[pos / B];
-      if (phys >= 0 && phys < p.num_blocks) {
-        constexpr int kChunks = D * S::kEsz / 16;  // 16-byte pieces of one row
-        const int64_t src = (static_cast<int64_t>(b) * p.num_kv_heads + kvh) * D;
-        const int64_t dst = ((static_cast<int64_t>(phys) * p.num_kv_heads + kvh) * B + pos % B) * D;
-        for (int c = lane; c < 2 * kChunks; c += 32) {
-          const bool is_v = c >= kChunks;
-          const int cc = is_v ? c - kChunks : c;
-          const uint4 val = reinterpret_cast<const uint4*>(static_cast<const T*>(is_v ? p.v_new : p.k_new) + src)[cc];
-          reinterpret_cast<uint4*>(const_cast<T*>(is_v ? vc : kc) + dst)[cc] = val;
-        }
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-      } else if (lane == 0) {
-        set_error(p.err, PA_DEVERR_BLOCK_ID);
-      }
-    }
-    __syncthreads();
-  }
   const uint64_t policy = l2_evict_first_policy();
 
   // Block ids of this warp's tiles k = 32*c + lane (two ids per tile when B = 8).
@@ -395,6 +374,33 @@ decode_kernel(const DecodeParams p) {
   const int base_idx = scatter_base<S::kNV, S::kDG>(lane);
   const int my_head = base_idx / S::kTPL;
 
+  // ---- fused append: the CTA whose range holds position L-1 writes the
+  // sequence's newest K/V row (this KV head) into its slot before reading
+  // it. Only the warp that owns the tile holding L-1 (tiles are dealt to
+  // warps round-robin) writes it and only that warp ever reads it, so the
+  // other warps start their copies at once. Generic stores, then the proxy
+  // fence by every writing lane and a warp barrier, so that lane 0's bulk
+  // copies (async proxy) see the row.
+  if (p.k_new != nullptr && L > 0 && t_begin <= L - 1 && L - 1 < t_end &&
+      warp == ((L - 1 - t_begin) / kTile) % NW) {
+    const int pos = L - 1;
+    const int phys = bt[pos / B];
+    if (phys >= 0 && phys < p.num_blocks) {
+      constexpr int kChunks = D * S::kEsz / 16;  // 16-byte pieces of one row
+      const int64_t src = (static_cast<int64_t>(b) * p.num_kv_heads + kvh) * D;
+      const int64_t dst = ((static_cast<int64_t>(phys) * p.num_kv_heads + kvh) * B + pos % B) * D;
+      for (int c = lane; c < 2 * kChunks; c += 32) {
+        const bool is_v = c >= kChunks;
+        const int cc = is_v ? c - kChunks : c;
+        const uint4 val = reinterpret_cast<const uint4*>(static_cast<const T*>(is_v ? p.v_new : p.k_new) + src)[cc];
+        reinterpret_cast<uint4*>(const_cast<T*>(is_v ? vc : kc) + dst)[cc] = val;
+      }
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+    } else if (lane == 0) {
+      set_error(p.err, PA_DEVERR_BLOCK_ID);
+    }
+    __syncwarp();
+  }
   // ---- pipeline --------------------------------------------------------------
   const int prologue = my_tiles < STAGES ? my_tiles : STAGES;
   for (int k = 0; k < prologue; ++k) issue(k);
