@@ -14,7 +14,8 @@
 //   warps 0-7  softmax: warps w and w+4 own row block 32*(w%4).. (TMEM lanes);
 //              warp half h takes keys [64h, 64h+64) of every tile as its own
 //              online-softmax stream (own running max / sum, own TMEM O
-//              accumulator), writes its P (bf16/f16) to shared memory,
+//              accumulator), writes its P (bf16/f16) back into TMEM over
+//              the S columns it read,
 //              rescales its O when its max grows by more than 2^8; the two
 //              streams are joined by the log-sum-exp rule when O is written;
 //   warps 8,10 producers: TMA tensor copies of the Q tile (once) and of each
@@ -25,7 +26,8 @@
 //              and land as zeros);
 //   warp 9     MMA: one thread issues S = Q K^T into a double-buffered TMEM
 //              accumulator and O_h += P_h V_h per key half into two TMEM
-//              accumulators (M = 128, K = 16 per instruction), completions via tcgen05.commit
+//              accumulators, P_h read straight from TMEM (A operand in tensor
+//              memory; M = 128, K = 16 per instruction), completions via tcgen05.commit
 //              on mbarriers; it zeroes V rows past the context in the last
 //              partial page chunk before they reach the PV product.
 // Every mbarrier wait is bounded; a timeout sets PA_DEVERR_WAIT and the CTA
@@ -83,14 +85,12 @@ template <int D>
 struct Smem {
   static constexpr int kQ = kM * D * 2;   // D/64 atoms of [128 rows x 128 B]
   static constexpr int kKV = kN * D * 2;  // one K or V tile
-  static constexpr int kP = kM * kN * 2;  // two atoms of [128 rows x 128 B]
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + kQ;
   static constexpr int oV = oK + kStagesK * kKV;
-  static constexpr int oP = oV + kStagesV * kKV;
-  static constexpr int oBar = oP + kP;
-  // q_full, k_full/k_empty[SK], v_full/v_empty[SV], s_full[2], p_full[2], o_done[2]
-  static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 2 + 2 + 2;
+  static constexpr int oBar = oV + kStagesV * kKV;
+  // q_full, k_full/k_empty[SK], v_full/v_empty[SV], s_full[2], p_full[half][S buffer], o_done[half]
+  static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 2 + 4 + 2;
   static constexpr int oTmem = oBar + kNumBars * 8;
   // The epilogue's row-max / row-sum exchange reuses the Q tile, which no
   // MMA reads any more by then: [2 halves][128 rows] floats each.
@@ -148,6 +148,17 @@ __device__ inline void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc), "r"(0), "r"(0), "r"(0), "r"(0)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16, one CTA: A (M x K, K-major)
+// lives in TMEM, row i in lane i, two 16-bit elements per 32-bit column.
+__device__ inline void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc), "r"(0), "r"(0), "r"(0), "r"(0)
       : "memory");
 }
 
@@ -330,8 +341,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   uint64_t* v_full = k_empty + kStagesK;
   uint64_t* v_empty = v_full + kStagesV;
   uint64_t* s_full = v_empty + kStagesV;  // [2]
-  uint64_t* p_full = s_full + 2;  // [2]: one per key half
-  uint64_t* o_done = p_full + 2;  // [2]
+  // p_full[half][S buffer u]: P of tile 2n+u written (phase n), one barrier
+  // per buffer so that the softmax, which no longer waits for the previous
+  // PV before writing P, can never be two phases ahead of the MMA's wait.
+  uint64_t* p_full = s_full + 2;  // [2 halves][2 buffers]
+  uint64_t* o_done = p_full + 4;  // [2]: PV of a key half done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::oTmem);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -369,7 +383,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
     for (int h = 0; h < 2; ++h) {
-      mbar_init(&p_full[h], 4);
+      mbar_init(&p_full[2 * h], 4);
+      mbar_init(&p_full[2 * h + 1], 4);
       mbar_init(&o_done[h], 1);
     }
     fence_mbar_init();
@@ -387,7 +402,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const uint32_t tS0 = tmem, tS1 = tmem + kN;
   const uint32_t tO0 = tmem + 2 * kN, tO1 = tmem + 2 * kN + D;
 
-  const uint32_t sQ = sb + S::oQ, sK = sb + S::oK, sV = sb + S::oV, sP = sb + S::oP;
+  const uint32_t sQ = sb + S::oQ, sK = sb + S::oK, sV = sb + S::oV;
   const int32_t* bt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
 
   if (warp == kProducerWarp || warp == kVProducerWarp) {
@@ -473,14 +488,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       __syncwarp();
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        if (!wait_all(&p_full[h], k & 1)) return false;
+        if (!wait_all(&p_full[2 * h + (k & 1)], (k >> 1) & 1)) return false;
         tc_fence_after();
         if (lane == 0) {
+          // P of key half h sits in the first 32 columns of that half's S region
+          const uint32_t tP = ((k & 1) ? tS1 : tS0) + h * (kN / 2);
 #pragma unroll
           for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
-            const uint64_t ad = sw128_desc(sP + h * (kM * 128) + (kk % 4) * 32, 1, 64);
             const uint64_t bd = sw128_desc(sV + st * S::kKV + kk * 2048, (kN * 128) >> 4, 64);
-            tc_mma(h ? tO1 : tO0, ad, bd, kIdescO, (k > 0 || kk > 4 * h) ? 1u : 0u);
+            tc_mma_ts(h ? tO1 : tO0, tP + (kk % 4) * 8, bd, kIdescO, (k > 0 || kk > 4 * h) ? 1u : 0u);
           }
           tc_commit(&o_done[h]);
           if (h == 1) tc_commit(&v_empty[st]);
@@ -585,24 +601,25 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float2 pa2 = __fadd2_rn(__fadd2_rn(ps2[0], ps2[1]), __fadd2_rn(ps2[2], ps2[3]));
       l = l * alpha + (pa2.x + pa2.y);
       m = m_use;
-      if (j > 0) {  // PV(j-1) of this half must be done before P is overwritten or O touched
-        if (!wait_all(&o_done[half], (j - 1) & 1)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-      }
-#pragma unroll
-      for (int c = 0; c < HC / 8; ++c) {
-        const uint32_t off = half * (kM * 128) + (r / 8) * 1024 + (r % 8) * 128 + ((c ^ (r % 8)) * 16);
-        *reinterpret_cast<uint4*>(smem + S::oP + off) =
-            make_uint4(pk[c * 4 + 0], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
+      // P goes back into TMEM over the first 32 columns of the S values this
+      // warp just read (S buffer j&1; PV(j-2), the last reader of that buffer,
+      // was issued before S(j), and tcgen05 MMAs run in issue order).
+      {
+        const uint32_t tP = ((j & 1) ? tS1 : tS0) + lane_off + half * HC;
+        tmem_st32(tP, reinterpret_cast<const float*>(pk));
       }
       if (j > 0) {
         // tcgen05.ld/st are warp-collective: the whole warp takes this branch
-        // when any of its rows needs a rescale (the others multiply by 1).
+        // when any of its rows needs a rescale (the others multiply by 1). O
+        // may be touched only once PV(j-1) of this half is done.
         const bool need = rescale && alpha != 1.f;
         if (__any_sync(0xffffffffu, need)) {
+          if (!wait_all(&o_done[half], (j - 1) & 1)) {
+            tmem_wait_st();
+            ok = false;
+            break;
+          }
+          tc_fence_after();
           const float f = need ? alpha : 1.f;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -613,13 +630,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             for (int e = 0; e < 32; ++e) o[e] *= f;
             tmem_st32(tO + c * 32, o);
           }
-          tmem_wait_st();
         }
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[half]);
+      if (lane == 0) mbar_arrive(&p_full[2 * half + (j & 1)]);
     }
     // epilogue: join the two halves, out = (O0 f0 + O1 f1) / (l0 f0 + l1 f1)
     bool got = ok;
