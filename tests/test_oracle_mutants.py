@@ -3,7 +3,8 @@
 Each mutant swaps one oracle function for a copy with one plausible slip in
 it: a dropped scale, a wrong KV head, pages in the wrong order, an off-by-one
 causal limit, a sign error, a merge that forgets a weight, a slot formula with
-block and offset swapped, a cache write one row off. The real oracle passes
+block and offset swapped, a cache write one row off, a merge in the wrong log
+base, a slot that skips the block table, K and V swapped. The real oracle passes
 every pin (tests/test_oracle.py); a pin set that let any of these through would
 not be pinning the oracle.
 """
@@ -104,7 +105,39 @@ _orig_copy = P.copy_blocks
 def copy_blocks_shifted(dst_k, dst_v, src_k, src_v, src_ids, dst_ids):
     return _orig_copy(dst_k, dst_v, src_k, src_v, [(int(s) + 1) % src_k.shape[0] for s in src_ids], dst_ids)
 
+def merge_exp2_units(part_o, part_m, part_l):
+    """Weights 2^(m_p - M) although m_p is in natural-log units (a units mix-up)."""
+    o, m, l = (np.asarray(x, dtype=np.float64) for x in (part_o, part_m, part_l))
+    N, H, NP, D = o.shape
+    out = np.zeros((N, H, D))
+    for b in range(N):
+        for h in range(H):
+            live = [p for p in range(NP) if l[b, h, p] > 0]
+            if not live:
+                continue
+            M = max(m[b, h, p] for p in live)
+            w = [2.0 ** (m[b, h, p] - M) for p in live]
+            out[b, h] = sum(wi * o[b, h, p] for wi, p in zip(w, live)) / sum(wi * l[b, h, p] for wi, p in zip(w, live))
+    return out
+
+
+def slots_ignore_table(block_tables, seq_idx, positions, block_size):
+    """Logical position used as the slot, block table skipped."""
+    out = np.full(len(seq_idx), -1, dtype=np.int64)
+    for i, (b, p) in enumerate(zip(np.asarray(seq_idx).tolist(), np.asarray(positions).tolist())):
+        if b >= 0:
+            out[i] = p
+    return out
+
+
+def cache_write_swaps_kv(k_new, v_new, k_cache, v_cache, slots):
+    return _orig_rc(v_new, k_new, k_cache, v_cache, slots)
+
+
 MUTANTS = {
+    "merge_exp2_units": ("merge", merge_exp2_units),
+    "slots_ignore_table": ("slot_mapping", slots_ignore_table),
+    "cache_write_swaps_kv": ("reshape_and_cache", cache_write_swaps_kv),
     "pages_reversed": ("gather_sequence", gather_pages_reversed),
     "wrong_kv_head": ("gather_sequence", gather_wrong_head),
     "row_offset": ("gather_sequence", gather_row_offset),
