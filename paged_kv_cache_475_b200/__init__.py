@@ -92,6 +92,9 @@ def _need(t: torch.Tensor, name: str, dtype=None, dim=None):
         raise TypeError(f"{name} must be a torch.Tensor")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}; the kernels run on the current device cuda:"
+                         f"{torch.cuda.current_device()}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
@@ -155,6 +158,8 @@ def pa_copy_blocks(dst_k, dst_v, src_k, src_v, src_block_ids, dst_block_ids, str
             raise ValueError(f"{n} must be a contiguous [P, Hkv, B, D] tensor")
         if not (t.is_cuda or t.is_pinned()):
             raise ValueError(f"{n} must be a CUDA tensor or pinned host memory")
+        if t.is_cuda and t.device.index != torch.cuda.current_device():
+            raise ValueError(f"{n} is on {t.device}, not on the current device")
     for n, t in (("src_block_ids", src_block_ids), ("dst_block_ids", dst_block_ids)):
         if t.dtype != torch.int32 or t.dim() != 1 or not (t.is_cuda or t.is_pinned()):
             raise ValueError(f"{n} must be int32 [n], on the GPU or pinned")

@@ -128,3 +128,22 @@ def test_copy_blocks_and_append_reject_bad_args_on_host(lib):
     assert lib.pa_decode_append(*args) == -1                       # k_new missing
     args[2] = ctypes.c_void_p(24)
     assert lib.pa_decode_append(*args) == -7                       # k_new misaligned
+
+
+def test_binding_rejects_host_tensors_before_any_launch():
+    """The Python layer refuses tensors the kernels could not address: no CPU fallback, no launch."""
+    import torch
+
+    import paged_kv_cache_475_b200 as pa
+    q = torch.zeros(2, 8, 128, dtype=torch.float16)
+    kc = torch.zeros(4, 2, 16, 128, dtype=torch.float16)
+    bt = torch.zeros(2, 4, dtype=torch.int32)
+    lens = torch.ones(2, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        pa.pa_decode(torch.empty_like(q), q, kc, kc.clone(), bt, lens, 0.1)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        pa.pa_reshape_and_cache(torch.zeros(1, 2, 128, dtype=torch.float16), torch.zeros(1, 2, 128, dtype=torch.float16),
+                                kc, kc.clone(), torch.zeros(1, dtype=torch.int64))
+    with pytest.raises(ValueError, match="pinned"):
+        pa.pa_copy_blocks(kc, kc.clone(), kc, kc.clone(), torch.zeros(1, dtype=torch.int32),
+                          torch.zeros(1, dtype=torch.int32))
