@@ -63,6 +63,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the cpu_baseline sample")
+    ap.add_argument("--reference-seconds", type=float, default=100.0,
+                    help="budget of the whole --impl reference run (sets its sample size)")
     a = ap.parse_args()
     a.warmup = max(a.warmup, 3)
     return a
@@ -316,7 +318,7 @@ def run_reference(args):
         return
     prefill = args.workload == "prefill_chunk"
     batch = make_workload(args.workload, args.block_size)
-    per_step_budget = max(0.2, 100.0 / (args.steps + args.warmup))
+    per_step_budget = max(0.05, args.reference_seconds / (args.steps + args.warmup))
     # one sample size sized to the per-step budget
     import oracle
     import workloads as W
