@@ -6,7 +6,6 @@ prefill on sampled output rows, which the oracle computes one by one. Pools
 are NaN-poisoned outside what each sequence may read.
 """
 import pytest
-import torch
 
 import oracle
 import workloads as W
