@@ -147,3 +147,49 @@ def test_binding_rejects_host_tensors_before_any_launch():
     with pytest.raises(ValueError, match="pinned"):
         pa.pa_copy_blocks(kc, kc.clone(), kc, kc.clone(), torch.zeros(1, dtype=torch.int32),
                           torch.zeros(1, dtype=torch.int32))
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "pa.h"
+
+int main(void) {
+  int fails = 0;
+  /* status strings, version, partition count */
+  if (strcmp(pa_status_string(PA_OK), "PA_OK") != 0) fails++;
+  if (pa_version() < 100) fails++;
+  if (pa_splitkv_num_partitions(100000, 512) != 196) fails++;
+  /* host-side checks run before any device work */
+  char fake[256];
+  if (pa_decode(fake, fake, fake, fake, (const int32_t*)fake, 4, (const int32_t*)fake, 2, 8, 2, 96, 16, 10,
+                0.1f, PA_F16, NULL) != PA_ERR_UNSUPPORTED) fails++;
+  if (pa_decode(fake, NULL, fake, fake, (const int32_t*)fake, 4, (const int32_t*)fake, 2, 8, 2, 128, 16, 10,
+                0.1f, PA_F16, NULL) != PA_ERR_NULL) fails++;
+  if (pa_prefill_chunk(fake, fake, fake, fake, (const int32_t*)fake, 4, (const int32_t*)fake, 2, 8, 8, 2, 128,
+                       16, 10, 0.1f, PA_F32, NULL) != PA_ERR_DTYPE) fails++;
+  if (pa_reshape_and_cache(NULL, NULL, NULL, NULL, NULL, 0, 10, 8, 128, 16, PA_F16, NULL) != PA_OK) fails++;
+  printf("fails=%d\n", fails);
+  return fails;
+}
+"""
+
+
+def test_header_compiles_as_c_and_links(lib, tmp_path):
+    """The boundary is a C ABI: pa.h compiles as C99, a C program links libpa.so and gets the host-side
+    status codes (no device work is started by these calls)."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi_check.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "abi_check"
+    libdir = os.path.join(ROOT, "paged_kv_cache_475_b200")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o",
+                    str(exe), "-L", libdir, "-lpa", f"-Wl,-rpath,{libdir}"], check=True, capture_output=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "fails=0" in r.stdout
