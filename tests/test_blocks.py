@@ -82,3 +82,59 @@ def test_tables_tensor_padding():
     m.allocate(1, 1)
     t = m.tables_tensor([0, 1])
     assert t.shape == (2, 3) and t[1, 1:].tolist() == [-1, -1]
+
+
+def test_random_operation_sequences_keep_the_invariants():
+    """Random allocate / fork / append / free sequences against a model of each sequence's tokens: the
+    reference counts always equal the table references, a token's slot never moves, two live
+    sequences never write the same slot, and a copy-on-write pair always copies the block the
+    sequence was reading into a private one."""
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    ops = st.lists(st.tuples(st.sampled_from(["alloc", "fork", "append", "free"]), st.integers(0, 7),
+                             st.integers(0, 7), st.integers(0, 70)), max_size=60)
+
+    @settings(max_examples=150, deadline=None)
+    @given(ops)
+    def run(seq_ops):
+        B = 8
+        m = BlockManager(48, B)
+        content = {}   # seq -> list of (physical block, offset) of its tokens, logical order
+        for op, a, b, n in seq_ops:
+            try:
+                if op == "alloc" and a not in m.tables:
+                    m.allocate(a, n)
+                    t = m.block_table(a)
+                    content[a] = [(t[p // B], p % B) for p in range(n)]
+                elif op == "fork" and a in m.tables and b not in m.tables:
+                    m.fork(a, b)
+                    content[b] = list(content[a])
+                elif op == "append" and a in m.tables:
+                    before = list(content[a])
+                    slot, pair = m.append_slot(a)
+                    t = m.block_table(a)
+                    pos = len(before)
+                    assert slot == t[pos // B] * B + pos % B
+                    if pair is not None:
+                        src, dst = pair
+                        assert src != dst and m.refcount[dst] == 1 and t[pos // B] == dst
+                        # the tokens already in the copied block move to the private copy
+                        before = [(dst if blk == src and i // B == pos // B else blk, off)
+                                  for i, (blk, off) in enumerate(before)]
+                    content[a] = before + [(slot // B, slot % B)]
+                    # no other live sequence may own the slot just written
+                    for s, toks in content.items():
+                        if s != a:
+                            assert (slot // B, slot % B) not in toks
+                elif op == "free" and a in m.tables:
+                    m.free(a)
+                    del content[a]
+            except OutOfBlocks:
+                pass
+            m.check()
+            for s, toks in content.items():
+                t = m.block_table(s)
+                assert [(t[i // B], i % B) for i in range(len(toks))] == toks
+
+    run()
