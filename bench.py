@@ -6,12 +6,20 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 A step is one pass of the hot path over one batch: map the step's new tokens
 to cache slots, write their K/V rows into the paged cache, then attend
-(single-pass decode, or split-KV + merge, or the chunked prefill). The default
+(single-pass decode, or split-KV + merge, or the chunked prefill). The headline
 workload is the Llama-3-8B-shaped single-layer decode (64 sequences, 32 q / 8
 KV heads, head dim 128, block size 16, context lengths uniform in
 [512, 4096], fp16). Inputs are synthetic and resident in HBM before timing;
 the KV read per step (~0.6 GB) is larger than the 126 MB L2, so no flush is
 needed between steps.
+
+A default run (one GPU) also times the other workloads with the same K and W
+and puts them in a "workloads" object of the same JSON line: the 4 x 100k
+split-KV decode, the 256-sequence chat trace (shared-prefix cascade, with the
+block-size sweep 8..128) and the bf16 chunked prefill. Each entry (and the
+headline) carries its roofline, end-to-end figure, and the clocks of its timed
+region, plus a "sustained" run of the same step for about two seconds whose
+clock record has enough samples under load to mean something.
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own batch
 (weak scaling, no collective on the data path); the step time is the max
@@ -61,11 +69,18 @@ def parse():
     ap.add_argument("--partition", default="auto")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the cpu_baseline sample")
+    ap.add_argument("--cpu-seconds", type=float, default=16.0,
+                    help="budget of the cpu_baseline samples (half with every core, half with one)")
+    ap.add_argument("--sustain-seconds", type=float, default=2.0,
+                    help="length of the extra run of each step that the clock record samples")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only --workload (by default the Llama decode line also carries the long-context, "
+                         "chat-trace (with the block-size sweep) and prefill workloads)")
     ap.add_argument("--reference-seconds", type=float, default=100.0,
                     help="budget of the whole --impl reference run (sets its sample size)")
     a = ap.parse_args()
     a.warmup = max(a.warmup, 3)
+    a.all_workloads = not a.headline_only and int(os.environ.get("WORLD_SIZE", "1")) == 1
     return a
 
 
@@ -131,13 +146,14 @@ def source_hash(files):
 
 
 class ClockSampler:
-    """nvidia-smi samples (every 200 ms) of SM clock and throttle reasons around the timed region.
+    """nvidia-smi samples (every 200 ms) of SM clock and throttle reasons around timed regions.
 
-    Each sample carries nvidia-smi's own timestamp. stop() keeps the samples
-    that fall inside the timed region (widened by one sampling period on each
-    side, so that a timed region shorter than the period still gets the
-    samples that bracket it) and waits, up to a second, for the first sample
-    after the region so that one always exists.
+    Each sample carries nvidia-smi's own timestamp. summary(t0, t1) keeps the
+    samples that fall inside one region (widened by one sampling period on
+    each side, so that a region shorter than the period still gets the samples
+    that bracket it), after waiting up to a second for the first sample after
+    the region so that one always exists. mark() names the region stop()
+    summarises.
     """
 
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -183,20 +199,13 @@ class ClockSampler:
         """Host wall-clock bounds of the timed region (time.time() before its first launch, after its sync)."""
         self.window = (t0, t1)
 
-    def stop(self):
+    def summary(self, t0, t1):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
-        t0, t1 = self.window if self.window else (0.0, float("inf"))
         deadline = time.time() + 1.0
         while time.time() < deadline and not any(r[0] >= t1 for r in self._rows()):
             time.sleep(0.05)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
         rows = self._rows()
-        os.unlink(self.f.name)
         inside = [r for r in rows if t0 - self.PERIOD_S <= r[0] <= t1 + self.PERIOD_S]
         if not inside:  # the sample nearest the region
             inside = sorted(rows, key=lambda r: min(abs(r[0] - t0), abs(r[0] - t1)))[:1]
@@ -206,6 +215,22 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max((r[2] for r in inside),
                                                                                      default=None),
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+    def stop(self):
+        t0, t1 = self.window if self.window else (0.0, float("inf"))
+        out = self.summary(t0, t1)
+        self.close()
+        return out
+
+    def close(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            os.unlink(self.f.name)
+            self.proc = None
 
 
 def dist_init(args):
@@ -276,36 +301,95 @@ def oracle_sample(batch, n_seqs):
     return s
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+
+    return platform.processor() or "unknown"
+
+
+def usable_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+class host_threads:
+    """Caps the host threads the oracle may use (BLAS pools and torch's intra-op pool) inside a with block."""
+
+    def __init__(self, n):
+        self.n = n
+
+    def __enter__(self):
+        import torch
+
+        self.torch_prev = torch.get_num_threads()
+        torch.set_num_threads(self.n)
+        try:
+            from threadpoolctl import threadpool_limits
+
+            self.ctl = threadpool_limits(limits=self.n)
+        except Exception:  # noqa: BLE001
+            self.ctl = None
+        return self
+
+    def __exit__(self, *exc):
+        import torch
+
+        torch.set_num_threads(self.torch_prev)
+        if self.ctl is not None:
+            self.ctl.restore_original_limits()
+
+
 def time_oracle(batch_cpu, budget_s, prefill=False):
     """Run the oracle step on growing samples until the budget is spent; returns (bytes_or_flops/s, info)."""
     import oracle
     import workloads as W
 
-    try:
-        from threadpoolctl import threadpool_info
-
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:  # noqa: BLE001
-        cores = os.cpu_count() or 1
     n = 1
     done_units, spent, seqs_done, steps = 0.0, 0.0, 0, 0
     while spent < budget_s and n <= batch_cpu.num_seqs:
         s = oracle_sample(batch_cpu, n)
         t0 = time.perf_counter()
+        oracle.step(s)
+        dt = time.perf_counter() - t0
         if prefill:
-            oracle.step(s)
             units = W.prefill_flops(s.context_lens.tolist(), s.chunk, s.num_q_heads, s.head_dim)
         else:
-            oracle.step(s)
             units = W.decode_kv_bytes(s.context_lens.tolist(), s.num_kv_heads, s.head_dim, s.k_cache.element_size())
-        dt = time.perf_counter() - t0
         done_units += units
         spent += dt
         seqs_done += n
         steps += 1
         if dt * 2 < budget_s - spent:
             n = min(batch_cpu.num_seqs, n * 2)
-    return done_units / spent, dict(cores=cores, seconds=round(spent, 2), seqs=seqs_done, samples=steps)
+    return done_units / spent, dict(seconds=round(spent, 2), seqs=seqs_done, samples=steps)
+
+
+def cpu_baseline(batch_cpu, budget_s, prefill, scale, unit):
+    """The oracle as it stands, on the host: with every usable core, then with one."""
+    cores = usable_cores()
+    with host_threads(cores):
+        v_all, info_all = time_oracle(batch_cpu, budget_s / 2, prefill)
+    with host_threads(1):
+        v_one, info_one = time_oracle(batch_cpu, budget_s / 2, prefill)
+    return {
+        "value": v_all / scale, "unit": unit, "cores": cores, "kind": "oracle",
+        "all_cores": {"value": v_all / scale, "threads": cores, **info_all},
+        "one_core": {"value": v_one / scale, "threads": 1, **info_one},
+        "cpu_model": cpu_model(), "cpu_count": os.cpu_count(),
+        "sample": "fp64 numpy oracle step (append + attention) on the first 1, 2, 4, ... sequences of the same "
+                  f"batch: {info_all['seqs']} sequences in {info_all['seconds']} s with {cores} threads (BLAS and "
+                  f"torch pools), {info_one['seqs']} in {info_one['seconds']} s with 1. The oracle's per-row "
+                  "matrix-vector loop is mostly single-threaded, so the two figures are close.",
+    }
 
 
 def run_reference(args):
@@ -345,18 +429,16 @@ def run_reference(args):
         units = W.decode_kv_bytes(sample.context_lens.tolist(), sample.num_kv_heads, sample.head_dim,
                                   sample.k_cache.element_size())
         value, unit = units * args.steps / dt / 1e9, "GB/s"
-    try:
-        from threadpoolctl import threadpool_info
+    import torch as _t
 
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:  # noqa: BLE001
-        cores = os.cpu_count() or 1
+    threads = _t.get_num_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": WORKLOAD_DESC[args.workload], "block_size": args.block_size},
-        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                         "cpu_model": cpu_model(), "cpu_count": os.cpu_count(),
                          "sample": f"first {n} of {batch.num_seqs} sequences per step, fp64 numpy"},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -367,27 +449,31 @@ def run_reference(args):
 # GPU side
 # ---------------------------------------------------------------------------
 
-def run_ours(args):
+def measure(name, block_size, partition_arg, K, W, rank, world, sampler, do_e2e=True, sustain_s=2.0,
+            cpu_budget_s=0.0):
+    """Time one workload's step: K steps (the reported value), a ~sustain_s run of the same step for the
+    clock record, and K end-to-end steps from host buffers. Returns the fields of its JSON entry."""
     import torch
 
-    world, rank, local = dist_init(args)
     import paged_kv_cache_475_b200 as pa
+    import workloads as Wl
     from paged_kv_cache_475_b200.step import DecodeStep, PrefillStep
 
-    prefill = args.workload == "prefill_chunk"
-    batch_cpu = make_workload(args.workload, args.block_size, seed_offset=100 * rank)
+    prefill = name == "prefill_chunk"
+    batch_cpu = make_workload(name, block_size, seed_offset=100 * rank)
     batch = batch_cpu.to("cuda")
-    esz = batch.k_cache.element_size()
     acct = workload_bytes(batch_cpu)
+    part = None
+    sp = None
     if prefill:
         step = PrefillStep(batch.num_seqs, batch.chunk, batch.num_q_heads, batch.head_dim, batch.q.dtype,
                            num_new_tokens=batch.new_seq.shape[0])
         partition = None
     else:
-        part = "auto" if args.partition == "auto" else (None if args.partition == "none" else int(args.partition))
+        part = "auto" if partition_arg == "auto" else (None if partition_arg == "none" else int(partition_arg))
         # chat trace: half the batch shares a 1024-token prompt -> the shared-prefix cascade
         sp = (batch_cpu.info["shared_prefix_tokens"], batch_cpu.info["shared_group"]) \
-            if args.workload == "chat_trace" and args.partition == "auto" else None
+            if name == "chat_trace" and partition_arg == "auto" else None
         step = DecodeStep(batch.num_seqs, batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
                           int(batch_cpu.context_lens.max()), batch.q.dtype,
                           num_new_tokens=batch.new_seq.shape[0], partition=part, shared_prefix=sp)
@@ -396,10 +482,8 @@ def run_ours(args):
     args_step = (batch.q, batch.k_new, batch.v_new, batch.k_cache, batch.v_cache, batch.block_tables,
                  batch.context_lens, batch.new_seq, batch.new_pos, batch.scale)
 
-    # The step, with CUDA events around the dominant kernel (on the current stream, where it runs).
     fused = (not prefill) and step.fused
     cascade = (not prefill) and getattr(step, "shared_prefix", None) is not None
-
     # A step that is one launch (or the cascade's fixed sequence) is timed by
     # one event at its end; its duration is the interval from the previous
     # step's end event (the timed region's start for the first step), which
@@ -448,15 +532,13 @@ def run_ours(args):
         if partition and not prefill:
             pa.pa_merge(step.out, step.part_o, step.part_m, step.part_l, batch.context_lens, partition)
 
-    sampler = ClockSampler(local)
-    sampler.start()
-    for _ in range(args.warmup):
+    for _ in range(W):
         run_step()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
 
-    K = args.steps
+    # ---- the K timed steps ----------------------------------------------------
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     w0 = time.time()
@@ -465,47 +547,54 @@ def run_ours(args):
         run_step(evs[i])
     t_end.record(stream)
     torch.cuda.synchronize()
-    sampler.mark(w0, time.time())
+    w1 = time.time()
     barrier(world)
     torch.cuda.synchronize()
-    clocks = sampler.stop()
-
-    ms_total = t_start.elapsed_time(t_end)
-    ms_total_max = max_over_ranks(ms_total, world)
-    ms_step = ms_total_max / K
+    ms_step = max_over_ranks(t_start.elapsed_time(t_end), world) / K
     if end_only:
         ends = [t_start] + [b for _, b in evs]
         kern_ms = statistics.mean(ends[i].elapsed_time(ends[i + 1]) for i in range(K))
     else:
         kern_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    # ---- the same step for ~sustain_s, so the clock record has samples under load
+    n_sus = int(min(200000, max(K, sustain_s / max(ms_step / 1e3, 1e-6))))
+    n_sus = int(max_over_ranks(n_sus, world))
+    s_start, s_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    s0 = time.time()
+    s_start.record(stream)
+    for _ in range(n_sus):
+        run_step()
+    s_end.record(stream)
+    torch.cuda.synchronize()
+    s1 = time.time()
+    barrier(world)
+    ms_sus = max_over_ranks(s_start.elapsed_time(s_end), world) / n_sus
     flags = pa.pa_read_error_flags(clear=True)
 
     hbm_peak, tf_peak, peak_src = measured_peaks()
     if prefill:
-        import workloads as W
-
-        flops = W.prefill_flops(batch_cpu.context_lens.tolist(), batch.chunk, batch.num_q_heads, batch.head_dim)
-        units_rank = flops
-        value = sum_over_ranks(flops, world) / (ms_step / 1e3) / 1e12
-        unit = "TFLOP/s"
+        flops = Wl.prefill_flops(batch_cpu.context_lens.tolist(), batch.chunk, batch.num_q_heads, batch.head_dim)
+        units_rank, scale, unit = flops, 1e12, "TFLOP/s"
         achieved = flops / (kern_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": tf_peak, "unit": "TFLOP/s",
                 "frac": achieved / tf_peak, "traffic": kernel_traffic("prefill_chunk"),
                 "peak_source": f"{peak_src} bf16 burst (cuBLAS)", "kernel": "pa_prefill_chunk",
-                "kernel_ms": kern_ms}
+                "kernel_ms": kern_ms, "algorithmic_flops_per_launch": flops}
     else:
-        units_rank = acct["kv_logical"]
-        value = sum_over_ranks(units_rank, world) / (ms_step / 1e3) / 1e9
-        unit = "GB/s"
+        units_rank, scale, unit = acct["kv_logical"], 1e9, "GB/s"
         kname = ("pa_decode_shared_prefix" if cascade else
                  ("pa_decode_splitkv_append" if partition else "pa_decode_append") if fused else
                  ("pa_decode_splitkv" if partition else "pa_decode"))
         attend_bytes = acct["attend_unique"] + (acct["append"] if fused else 0)
         achieved = attend_bytes / (kern_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": kernel_traffic(f"{kname}:{args.workload}:B{args.block_size}"),
+                "frac": achieved / hbm_peak, "traffic": kernel_traffic(f"{kname}:{name}:B{block_size}"),
                 "peak_source": f"{peak_src} HBM copy bandwidth", "kernel": kname, "kernel_ms": kern_ms,
                 "algorithmic_bytes_per_launch": attend_bytes}
+    value = sum_over_ranks(units_rank, world) / (ms_step / 1e3) / scale
 
     # ---- end to end: host buffers in, result out, through the C ABI -----------
     # Every step uploads its inputs (q, the new K/V rows, block tables, context
@@ -516,7 +605,7 @@ def run_ours(args):
     # buffers), and events order every buffer's reuse. The inputs travel as one
     # packed staging buffer (one upload per step).
     e2e = None
-    if not args.no_e2e:
+    if do_e2e:
         templates = [batch.q, batch.k_new, batch.v_new, batch.block_tables, batch.context_lens, batch.new_seq,
                      batch.new_pos]
         offs, off = [], 0
@@ -571,7 +660,7 @@ def run_ours(args):
                 host_out[s].copy_(out, non_blocking=True)
             ev_down[s].record(down)
 
-        for i in range(args.warmup):
+        for i in range(W):
             e2e_step(i)
         torch.cuda.synchronize()
         barrier(world)
@@ -586,43 +675,110 @@ def run_ours(args):
         torch.cuda.synchronize()
         barrier(world)
         ms_e2e = max_over_ranks(e0.elapsed_time(e1), world) / K
-        e2e_val = sum_over_ranks(units_rank, world) / (ms_e2e / 1e3) / (1e12 if prefill else 1e9)
-        e2e = {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": ms_e2e, "transfers": "overlapped with compute (separate copy streams, double-buffered)"}
+        e2e = {"value": sum_over_ranks(units_rank, world) / (ms_e2e / 1e3) / scale, "unit": unit,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+               "transfers": "overlapped with compute (separate copy streams, double-buffered)"}
+        flags |= pa.pa_read_error_flags(clear=True)
 
-    # ---- CPU baseline: the oracle on a bounded sample, rank 0 at N = 1 ---------
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, info = time_oracle(batch_cpu, args.cpu_seconds, prefill)
-        cpu = {"value": v / (1e12 if prefill else 1e9), "unit": unit, "cores": info["cores"], "kind": "oracle",
-               "sample": f"fp64 numpy oracle step (append + attention) on the first 1,2,4,.. sequences of the "
-                         f"same batch; {info['seqs']} sequences over {info['samples']} runs in {info['seconds']} s"}
+    if cpu_budget_s > 0 and rank == 0 and world == 1:
+        cpu = cpu_baseline(batch_cpu, cpu_budget_s, prefill, scale, unit)
+
+    res = {
+        "value": value, "unit": unit, "ms_per_step": ms_step, "steps": K, "warmup": W,
+        "dtype": batch_cpu.info["dtype"],
+        "config": {
+            "workload": WORKLOAD_DESC[name], "num_seqs": batch.num_seqs, "block_size": batch.block_size,
+            "head_dim": batch.head_dim, "num_q_heads": batch.num_q_heads, "num_kv_heads": batch.num_kv_heads,
+            "partition": partition, "fused_append": fused,
+            "shared_prefix": list(step.shared_prefix) if cascade else None,
+            "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush" if not cascade else
+                  "unique KV (522 MB) larger than L2, no flush; the shared prefix is read once per step by design",
+            "kv_bytes_logical_per_rank": acct["kv_logical"], "kv_bytes_unique_per_rank": acct["kv_unique"],
+            "parallelism": f"dp{world} (independent batches per GPU)",
+        },
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": step.launches_per_call * K,
+        "sustained": {"steps": n_sus, "ms_per_step": ms_sus,
+                      "value": sum_over_ranks(units_rank, world) / (ms_sus / 1e3) / scale, "unit": unit},
+        "device_error_flags": flags,
+        "_windows": {"timed": (w0, w1), "sustained": (s0, s1)},
+    }
+    if cpu is not None:
+        res["cpu_baseline"] = cpu
+    if not prefill:
+        res["seq_steps_per_s"] = batch.num_seqs * world / (ms_step / 1e3)
+        res["pct_of_peak"] = 100.0 * value / (hbm_peak * world)
+        if acct["kv_unique"] != acct["kv_logical"]:
+            res["unique_bytes_frac"] = acct["attend_unique"] / (ms_step / 1e3) / 1e9 / hbm_peak
+    del step, batch, args_step
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
+EXTRA_WORKLOADS = ("long_context", "chat_trace", "prefill_chunk")
+SWEEP_BLOCK_SIZES = (8, 16, 32, 64, 128)
+
+
+def run_ours(args):
+    import torch
+
+    world, rank, local = dist_init(args)
+    sampler = ClockSampler(local)
+    sampler.start()
+    K, W = args.steps, args.warmup
+    main = measure(args.workload, args.block_size, args.partition, K, W, rank, world, sampler,
+                   do_e2e=not args.no_e2e, sustain_s=args.sustain_seconds,
+                   cpu_budget_s=0.0 if args.no_cpu_baseline else args.cpu_seconds)
+    extras = {}
+    sweep = []
+    if args.all_workloads and args.workload == "llama_decode":
+        for name in EXTRA_WORKLOADS:
+            extras[name] = measure(name, 16, "auto", K, W, rank, world, sampler, do_e2e=not args.no_e2e,
+                                   sustain_s=args.sustain_seconds)
+        for B in SWEEP_BLOCK_SIZES:  # the pages' block-size question, on the chat trace (cascade)
+            r = measure("chat_trace", B, "auto", K, W, rank, world, sampler, do_e2e=False, sustain_s=0.0)
+            sweep.append({"block_size": B, "value": r["value"], "unit": r["unit"], "ms_per_step": r["ms_per_step"],
+                          "kernel_ms": r["roofline"]["kernel_ms"], "roofline_frac": r["roofline"]["frac"],
+                          "device_error_flags": r["device_error_flags"], "_windows": r["_windows"]})
+
+    def clocks_of(r):
+        win = r.pop("_windows")
+        r["clocks"] = sampler.summary(*win["timed"])
+        if "sustained" in win and "sustained" in r:
+            r["sustained"]["clocks"] = sampler.summary(*win["sustained"])
+        return r
+
+    clocks_of(main)
+    for r in extras.values():
+        clocks_of(r)
+    for r in sweep:
+        clocks_of(r)
+    sampler.close()
 
     if rank == 0:
-        launches = step.launches_per_call * K
         line = {
-            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K, "warmup": args.warmup,
-            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": {"f16": "f16", "bf16": "bf16", "f32": "f32"}[batch_cpu.info["dtype"]], "data": "synthetic",
-            "config": {
-                "workload": WORKLOAD_DESC[args.workload], "num_seqs": batch.num_seqs, "block_size": batch.block_size,
-                "head_dim": batch.head_dim, "num_q_heads": batch.num_q_heads, "num_kv_heads": batch.num_kv_heads,
-                "partition": partition, "fused_append": fused,
-                "shared_prefix": list(step.shared_prefix) if cascade else None,
-                "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
-                "kv_bytes_logical_per_rank": acct["kv_logical"], "kv_bytes_unique_per_rank": acct["kv_unique"],
-                "parallelism": f"dp{world} (independent batches per GPU)",
-            },
-            "roofline": roof,
-            "cpu_baseline": cpu,
-            "e2e": e2e,
-            "gpu_launches": launches,
-            "clocks": clocks,
-            "device_error_flags": flags,
+            "metric": METRIC, "value": main["value"], "unit": main["unit"], "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": main["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": main["dtype"], "data": "synthetic", "config": main["config"],
+            "roofline": main["roofline"], "cpu_baseline": main.get("cpu_baseline"), "e2e": main["e2e"],
+            "gpu_launches": main["gpu_launches"] + sum(r["gpu_launches"] for r in extras.values()),
+            "clocks": main["clocks"], "sustained": main["sustained"],
+            "device_error_flags": main["device_error_flags"],
         }
-        if not prefill:
-            line["seq_steps_per_s"] = batch.num_seqs * world / (ms_step / 1e3)
-            line["pct_of_peak"] = 100.0 * value / (hbm_peak * world)
+        for k in ("seq_steps_per_s", "pct_of_peak"):
+            if k in main:
+                line[k] = main[k]
+        if extras:
+            line["gpu_launches_headline"] = main["gpu_launches"]
+            line["workloads"] = {}
+            for name, r in extras.items():
+                r.pop("steps", None)
+                r.pop("warmup", None)
+                line["workloads"][name] = r
+            line["workloads"]["chat_trace"]["block_size_sweep"] = sweep
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist

@@ -177,8 +177,26 @@ PA_API int pa_decode_append(void* out, const void* q, const void* k_new, const v
                             int num_blocks, float scale, pa_dtype dtype, void* stream);
 
 /* Number of partitions of `partition_size` tokens a context of
- * max_context_len tokens needs (at least 1). */
+ * max_context_len tokens needs (at least 1; 0 if partition_size <= 0). */
 PA_API int pa_splitkv_num_partitions(int max_context_len, int partition_size);
+
+/*
+ * pa_splitkv_workspace_bytes - size of one caller-owned buffer that holds all
+ * three split-KV partial arrays of pa_decode_splitkv / pa_merge for N
+ * sequences, Hq query heads, head dim D, contexts of at most max_context_len
+ * tokens and partitions of partition_size tokens. With
+ * NP = pa_splitkv_num_partitions(max_context_len, partition_size) and every
+ * part rounded up to a multiple of 256 bytes, the buffer holds
+ *   part_o float [N, Hq, NP, D] at byte 0,
+ *   part_m float [N, Hq, NP]    at byte round256(N*Hq*NP*D*4),
+ *   part_l float [N, Hq, NP]    right after part_m, at round256(...) + round256(N*Hq*NP*4).
+ * (The split partials are the per-block sums of [FvP] eq. (4); the pages fix
+ * no memory layout for them.) Pure host arithmetic, no CUDA call. Returns 0
+ * when N == 0, when an argument is negative (N, max_context_len) or not
+ * positive (Hq, D, partition_size), or when the size does not fit in size_t.
+ */
+PA_API size_t pa_splitkv_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
+                                         int partition_size);
 
 /*
  * pa_decode_splitkv - per-partition online-softmax state of a decode step.
@@ -258,7 +276,10 @@ PA_API int pa_decode_splitkv_append(float* part_o, float* part_m, float* part_l,
  *   M = max_p m_p,  Lsum = sum_p exp(m_p - M) l_p,
  *   out[b,h,:] = sum_p exp(m_p - M) o_p / Lsum   (rounded to `dtype`)
  * A row with no such partition is zero. context_lens and partition_size
- * must be the ones given to pa_decode_splitkv.
+ * must be the ones given to pa_decode_splitkv: with them the merge reads only
+ * the ceil(L_b / S) partitions that hold tokens of row b and never touches
+ * the slots of partitions past a short row's context (the pages give no
+ * merge interface; this is the reading of the log-sum-exp rule used here).
  */
 PA_API int pa_merge(void* out, const float* part_o, const float* part_m, const float* part_l,
                     const int32_t* context_lens, int num_seqs, int num_q_heads, int head_dim,
@@ -299,10 +320,16 @@ PA_API int pa_prefill_chunk(void* out, const void* q, const void* k_cache, const
  * 256 bytes); larger requests return PA_ERR_WORKSPACE and launch nothing.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
- * capture begins. Every call on a device shares the one array: calls whose
- * kernels overlap on the GPU (other streams, other host threads) race and
- * must be serialised by the caller. Nothing in the array needs clearing: each
- * call writes every partial it later reads.
+ * capture begins. The address is remembered together with the CUDA context
+ * it was taken in: after cudaDeviceReset the array lives at a new address,
+ * and the next call on that device looks it up again (so make that call
+ * outside a stream capture too). Every call on a device shares the one
+ * array: calls whose kernels overlap on the GPU (other streams, other host
+ * threads) race and must be serialised by the caller. Nothing in the array
+ * needs clearing: each call writes every partial it later reads.
+ * N * Hq * num_partitions is checked against the array size before any
+ * product is formed, so no accepted shape can wrap the size arithmetic;
+ * num_partitions > 2^30 returns PA_ERR_SHAPE.
  */
 PA_API int pa_decode_splitkv_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
                                      const int32_t* block_tables, int max_blocks_per_seq,
@@ -327,7 +354,7 @@ PA_API const char* pa_last_cuda_error(void);
 /* Human-readable name of a pa_status value. */
 PA_API const char* pa_status_string(int status);
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor): 101 adds pa_splitkv_workspace_bytes. */
 PA_API int pa_version(void);
 
 #ifdef __cplusplus

@@ -17,8 +17,7 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-# PA_LIBRARY may point at another build of the same library (e.g. a tuning variant).
-LIB_PATH = os.environ.get("PA_LIBRARY") or os.path.join(_PKG, "libpa.so")
+LIB_PATH = os.path.join(_PKG, "libpa.so")  # the in-tree build, always
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python paged_kv_cache_475_b200/build.py`")
@@ -45,6 +44,7 @@ _SIGS = {
     "pa_decode_shared_prefix": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                                 _vp, _vp, _i, _f, _i, _vp],
     "pa_splitkv_num_partitions": [_i, _i],
+    "pa_splitkv_workspace_bytes": [_i, _i, _i, _i, _i],
     "pa_decode_splitkv": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                           _i, _vp],
     "pa_decode_splitkv_append": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i,
@@ -63,7 +63,7 @@ for _name, _args in _SIGS.items():
     _fn = getattr(_lib, _name)
     _fn.argtypes = _args
     _fn.restype = {"pa_status_string": ctypes.c_char_p, "pa_last_cuda_error": ctypes.c_char_p,
-                   "pa_noalloc_scratch_bytes": _sz}.get(_name, _i)
+                   "pa_noalloc_scratch_bytes": _sz, "pa_splitkv_workspace_bytes": _sz}.get(_name, _i)
 
 
 class PagedAttentionError(RuntimeError):
@@ -115,6 +115,13 @@ def version() -> int:
 
 def pa_splitkv_num_partitions(max_context_len: int, partition_size: int) -> int:
     return _lib.pa_splitkv_num_partitions(int(max_context_len), int(partition_size))
+
+
+def pa_splitkv_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int,
+                               partition_size: int) -> int:
+    """Bytes of one buffer holding part_o, part_m and part_l (layout in include/pa.h); 0 if invalid."""
+    return _lib.pa_splitkv_workspace_bytes(int(num_seqs), int(num_q_heads), int(head_dim), int(max_context_len),
+                                           int(partition_size))
 
 
 def pa_slot_mapping(slot_mapping, block_tables, seq_idx, positions, block_size: int, stream=None):
@@ -334,6 +341,26 @@ def pa_read_error_flags(clear: bool = True) -> int:
     v = ctypes.c_uint32(0)
     _check(_lib.pa_read_error_flags(ctypes.byref(v), 1 if clear else 0), "pa_read_error_flags")
     return v.value
+
+
+def splitkv_workspace(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int, partition_size: int,
+                      device="cuda"):
+    """(part_o, part_m, part_l) carved out of ONE caller-owned buffer of pa_splitkv_workspace_bytes bytes,
+    at the offsets include/pa.h gives (each part starts on a 256-byte boundary)."""
+    total = pa_splitkv_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len, partition_size)
+    if total == 0:
+        raise ValueError("invalid split-KV workspace shape")
+    NP = pa_splitkv_num_partitions(max_context_len, partition_size)
+    cells = num_seqs * num_q_heads * NP
+    o_bytes = (cells * head_dim * 4 + 255) // 256 * 256
+    ml_bytes = (cells * 4 + 255) // 256 * 256
+    if o_bytes + 2 * ml_bytes != total:
+        raise RuntimeError("pa_splitkv_workspace_bytes disagrees with the documented layout")
+    buf = torch.empty(total, dtype=torch.uint8, device=device)
+    part_o = buf[:cells * head_dim * 4].view(torch.float32).view(num_seqs, num_q_heads, NP, head_dim)
+    part_m = buf[o_bytes:o_bytes + cells * 4].view(torch.float32).view(num_seqs, num_q_heads, NP)
+    part_l = buf[o_bytes + ml_bytes:o_bytes + ml_bytes + cells * 4].view(torch.float32).view(num_seqs, num_q_heads, NP)
+    return part_o, part_m, part_l
 
 
 def splitkv_buffers(num_seqs: int, num_q_heads: int, head_dim: int, num_partitions: int, device="cuda"):

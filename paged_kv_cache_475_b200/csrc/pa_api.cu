@@ -1,4 +1,7 @@
-// Library-wide entry points: device error word, status strings, version.
+// Library-wide entry points: device error word, workspace sizes, status strings, version.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <cstdio>
 #include <mutex>
 
@@ -9,9 +12,32 @@ namespace pa {
 // One error word per device; kernels OR PA_DEVERR_* bits into it.
 __device__ unsigned int g_error_word;
 
+uint64_t current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return static_cast<uint64_t>(id);
+}
+
 namespace {
 constexpr int kMaxDevices = 64;
-unsigned int* g_err_ptr[kMaxDevices] = {};
+ContextCached<unsigned int*> g_err_ptr[kMaxDevices];
 std::mutex g_err_mu;
 }  // namespace
 
@@ -19,12 +45,12 @@ unsigned int* device_error_word() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lk(g_err_mu);
-  if (!g_err_ptr[dev]) {
+  if (!g_err_ptr[dev].valid()) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
-    g_err_ptr[dev] = static_cast<unsigned int*>(p);
+    g_err_ptr[dev].set(static_cast<unsigned int*>(p));
   }
-  return g_err_ptr[dev];
+  return g_err_ptr[dev].value;
 }
 
 namespace {
@@ -67,10 +93,22 @@ extern "C" PA_API const char* pa_status_string(int status) {
   }
 }
 
-extern "C" PA_API int pa_version(void) { return 100; }
+extern "C" PA_API int pa_version(void) { return 101; }
 
 extern "C" PA_API int pa_splitkv_num_partitions(int max_context_len, int partition_size) {
   if (partition_size <= 0) return 0;
   if (max_context_len <= 0) return 1;
-  return (max_context_len + partition_size - 1) / partition_size;
+  return static_cast<int>((static_cast<int64_t>(max_context_len) + partition_size - 1) / partition_size);
+}
+
+extern "C" PA_API size_t pa_splitkv_workspace_bytes(int num_seqs, int num_q_heads, int head_dim,
+                                                    int max_context_len, int partition_size) {
+  if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len < 0 || partition_size <= 0)
+    return 0;
+  const int np = pa_splitkv_num_partitions(max_context_len, partition_size);
+  pa::SplitkvLayout lay;
+  if (!pa::splitkv_layout(static_cast<size_t>(num_seqs) * static_cast<size_t>(num_q_heads),
+                          static_cast<size_t>(np), static_cast<size_t>(head_dim), &lay))
+    return 0;
+  return lay.total;
 }

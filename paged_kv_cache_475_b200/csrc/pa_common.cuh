@@ -17,6 +17,51 @@ namespace pa {
 // Device error word of the current device (lives in pa_api.cu).
 unsigned int* device_error_word();
 
+// Identity of the CUDA context current on this host thread, unique over the
+// life of the process; 0 when no context is current or the driver cannot say.
+// A device reset destroys the primary context and with it every address of a
+// module-scope __device__ variable and every function attribute set in it, so
+// per-device caches of those remember the context they were taken in.
+uint64_t current_context_id();
+
+// A per-device cached value, valid only in the context it was taken in.
+template <typename V>
+struct ContextCached {
+  uint64_t ctx = 0;
+  V value{};
+  bool valid() const {
+    const uint64_t now = current_context_id();
+    return now != 0 && now == ctx;
+  }
+  void set(V v) {
+    value = v;
+    ctx = current_context_id();
+  }
+};
+
+// Byte layout of a split-KV workspace holding part_o [rows, np, D] at offset
+// 0, part_m [rows, np] at o_bytes and part_l [rows, np] at o_bytes + ml_bytes
+// (rows = N * Hq), each part rounded up to a multiple of 256 bytes. Returns
+// false when a size does not fit in size_t.
+struct SplitkvLayout {
+  size_t o_bytes = 0, ml_bytes = 0, total = 0;
+};
+inline bool splitkv_layout(size_t rows, size_t np, size_t head_dim, SplitkvLayout* out) {
+  constexpr size_t kMax = ~size_t(0);
+  if (rows != 0 && np > kMax / rows) return false;
+  const size_t cells = rows * np;
+  const size_t row_bytes = head_dim * sizeof(float);
+  if (row_bytes != 0 && cells > (kMax - 255) / row_bytes) return false;
+  if (cells > (kMax - 255) / sizeof(float)) return false;
+  const size_t o = (cells * row_bytes + 255) & ~size_t(255);
+  const size_t ml = (cells * sizeof(float) + 255) & ~size_t(255);
+  if (ml > (kMax - o) / 2) return false;
+  out->o_bytes = o;
+  out->ml_bytes = ml;
+  out->total = o + 2 * ml;
+  return true;
+}
+
 // Shared-prefix mode of the tensor-core prefill kernel: the group's decode
 // queries attend to keys [0, prefix_len) of block-table row 0, cut into
 // key_splits ranges, and the results land as split-KV partials in slots

@@ -714,13 +714,14 @@ int launch_decode(const DecodeParams& prm, int grid_x, cudaStream_t stream) {
   constexpr int ST = (DecodeShape<T, D, G>::kTileBytes >= 8192 && kDecodeStages > 2) ? 2 : kDecodeStages;
   using M = DecodeSmem<T, D, G, NW, ST>;
   auto kern = decode_kernel<T, D, G, NW, ST>;
-  static bool attr_done[64] = {};
+  // The attribute lives in the context: set it again after a device reset.
+  static ContextCached<bool> attr_done[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+  if (dev < 0 || dev >= 64 || !attr_done[dev].valid()) {
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, M::kTotal);
     if (e != cudaSuccess) return record_cuda_error(e, "decode: set max dynamic shared memory");
-    attr_done[dev] = true;
+    if (dev >= 0 && dev < 64) attr_done[dev].set(true);
   }
   dim3 grid(grid_x, prm.num_kv_heads, prm.num_seqs);
   kern<<<grid, NW * 32, M::kTotal, stream>>>(prm);
@@ -1055,22 +1056,26 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
 static __device__ __align__(256) unsigned char g_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-static unsigned char* g_scratch_dev[kMaxDevices] = {};
+static ContextCached<unsigned char*> g_scratch_dev[kMaxDevices];
 static std::mutex g_scratch_mu;
 
 // Device address of g_scratch on the current device. In host code the name
 // g_scratch is only a host-side stand-in, so the address is looked up once per
-// device (with that device current) and cached.
+// device (with that device current) and cached together with the identity of
+// the context it was taken in: after a device reset the array lives at a new
+// address, and the next call looks it up again.
 static int scratch_address(unsigned char** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_dev[dev]) {
+  if (!g_scratch_dev[dev].valid()) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return PA_ERR_CUDA;
-    g_scratch_dev[dev] = static_cast<unsigned char*>(p);
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
+    if (e != cudaSuccess) return record_cuda_error(e, "noalloc: look up the scratch array's device address");
+    if (p == nullptr) return PA_ERR_CUDA;
+    g_scratch_dev[dev].set(static_cast<unsigned char*>(p));
   }
-  *out = g_scratch_dev[dev];
+  *out = g_scratch_dev[dev].value;
   return PA_OK;
 }
 
@@ -1090,19 +1095,24 @@ extern "C" PA_API int pa_decode_splitkv_noalloc(void* out, const void* q, const 
   if (st != PA_OK || num_seqs == 0) return st;
   if (!out) return PA_ERR_NULL;
   if (partition_size <= 0 || partition_size % kTile || num_partitions <= 0) return PA_ERR_WORKSPACE;
-  if (num_seqs > 65535) return PA_ERR_SHAPE;
-  // Partials: o [rows, NP, D], then m and l [rows, NP], each start 256-byte aligned.
-  const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads;
-  const size_t cells = rows * static_cast<size_t>(num_partitions);
-  const size_t o_bytes = (cells * head_dim * sizeof(float) + 255) & ~size_t(255);
-  const size_t ml_bytes = (cells * sizeof(float) + 255) & ~size_t(255);
-  if (o_bytes + 2 * ml_bytes > pa::noalloc::kNoAllocScratchBytes) return PA_ERR_WORKSPACE;
+  if (num_seqs > 65535 || num_partitions > (1 << 30)) return PA_ERR_SHAPE;
+  // Partials: o [rows, NP, D], then m and l [rows, NP], each start 256-byte
+  // aligned. The partition count is compared by division first, so that no
+  // product below can wrap around for any accepted shape.
+  const size_t rows = static_cast<size_t>(num_seqs) * static_cast<size_t>(num_q_heads);
+  const size_t cell_bytes = static_cast<size_t>(head_dim + 2) * sizeof(float);
+  if (static_cast<size_t>(num_partitions) > pa::noalloc::kNoAllocScratchBytes / (rows * cell_bytes))
+    return PA_ERR_WORKSPACE;
+  SplitkvLayout lay;
+  if (!splitkv_layout(rows, static_cast<size_t>(num_partitions), static_cast<size_t>(head_dim), &lay) ||
+      lay.total > pa::noalloc::kNoAllocScratchBytes)
+    return PA_ERR_WORKSPACE;
   unsigned char* base = nullptr;
   st = pa::noalloc::scratch_address(&base);
   if (st != PA_OK) return st;
   float* part_o = reinterpret_cast<float*>(base);
-  float* part_m = reinterpret_cast<float*>(base + o_bytes);
-  float* part_l = reinterpret_cast<float*>(base + o_bytes + ml_bytes);
+  float* part_m = reinterpret_cast<float*>(base + lay.o_bytes);
+  float* part_l = reinterpret_cast<float*>(base + lay.o_bytes + lay.ml_bytes);
   // Every partition p < num_partitions of every row is written by the split
   // pass (empty ones as m = -inf, l = 0, o = 0) before the merge reads it, so
   // nothing left in the array by an earlier call is ever read.

@@ -760,13 +760,14 @@ int launch(const Params& prm, const void* q, const void* k_cache, const void* v_
   // Above half of the SM's shared memory, so one CTA (and one TMEM allocation
   // of 512 columns) per SM.
   const int smem = Smem<D>::kAlloc > 120 * 1024 ? Smem<D>::kAlloc : 120 * 1024;
-  static bool attr_done[64] = {};
+  // The attribute lives in the context: set it again after a device reset.
+  static ContextCached<bool> attr_done[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+  if (dev < 0 || dev >= 64 || !attr_done[dev].valid()) {
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return record_cuda_error(e, "prefill: set max dynamic shared memory");
-    attr_done[dev] = true;
+    if (dev >= 0 && dev < 64) attr_done[dev].set(true);
   }
   dim3 grid((prm.chunk + QT - 1) / QT, prm.num_kv_heads, prm.prefix_len > 0 ? prm.key_splits : prm.num_seqs);
   kern<<<grid, kThreads, smem, stream>>>(mq, mk, mv, prm);

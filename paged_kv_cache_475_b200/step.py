@@ -13,7 +13,7 @@ import torch
 
 from . import (pa_decode, pa_decode_append, pa_decode_shared_prefix, pa_decode_splitkv,
                pa_decode_splitkv_append, pa_merge, pa_prefill_chunk, pa_reshape_and_cache, pa_slot_mapping,
-               pa_splitkv_num_partitions)
+               pa_splitkv_num_partitions, splitkv_workspace)
 
 NUM_SMS_B200 = 148
 
@@ -79,11 +79,10 @@ class DecodeStep:
         self.slot_mapping = torch.empty(T, dtype=torch.int64, device=device)
         self.out = torch.empty((num_seqs, num_q_heads, head_dim), dtype=dtype, device=device)
         if partition:
+            # one buffer sized by the library's own workspace query, carved into the three partial arrays
             self.num_parts = pa_splitkv_num_partitions(max_context_len, partition)
-            self.part_o = torch.empty((num_seqs, num_q_heads, self.num_parts, head_dim), dtype=torch.float32,
-                                      device=device)
-            self.part_m = torch.empty((num_seqs, num_q_heads, self.num_parts), dtype=torch.float32, device=device)
-            self.part_l = torch.empty_like(self.part_m)
+            self.part_o, self.part_m, self.part_l = splitkv_workspace(num_seqs, num_q_heads, head_dim,
+                                                                      max_context_len, partition, device)
         self.launches_per_call = (2 if partition else 1) if self.fused else (4 if partition else 3)
 
     def __call__(self, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, new_seq, new_pos,

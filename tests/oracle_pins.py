@@ -344,9 +344,69 @@ def pin_copy_blocks(P):
         assert torch.equal(ok_[d_].view(torch.int16), dk[d_].view(torch.int16))
 
 
+def pin_step_appends_then_attends(P):
+    """step(): the step's new rows land in their slots before attention reads them.
+
+    The pin appends on its own: for every new token t of sequence s at
+    position pos, the row (block_tables[s][pos // B], pos % B) of every KV head
+    takes k_new[t] / v_new[t] ([FvP] 内存管理机制, left-to-right fill; [FP]
+    PagedAttention steps 1-3). The slots those rows occupy are NaN-poisoned in
+    the input pools, so attending over the caches as they were before the
+    append gives NaN rows. step() must return those caches bit for bit, the
+    slots block * B + pos % B, and the attention of the appended caches.
+    """
+    for b in (small_decode(seed=111), small_prefill(seed=112), small_decode(seed=113, dtype="f16", B=8)):
+        out, kc, vc, slots = P.step(b)
+        B = b.block_size
+        kc2, vc2 = b.k_cache.clone(), b.v_cache.clone()
+        expect_slots = []
+        for t in range(b.new_seq.shape[0]):
+            s_, pos = int(b.new_seq[t]), int(b.new_pos[t])
+            blk = int(b.block_tables[s_][pos // B])
+            kc2[blk, :, pos % B] = b.k_new[t]
+            vc2[blk, :, pos % B] = b.v_new[t]
+            expect_slots.append(blk * B + pos % B)
+        assert list(np.asarray(slots).tolist()) == expect_slots
+        ib = torch.int32 if kc.dtype == torch.float32 else torch.int16
+        assert torch.equal(kc.view(ib), kc2.view(ib)) and torch.equal(vc.view(ib), vc2.view(ib))
+        assert np.isfinite(out).all()
+        ref = P.attention(b.q, kc2, vc2, b.block_tables, b.context_lens, b.scale)
+        assert np.array_equal(out, ref)
+
+
+def pin_step_partition_branch(P):
+    """step(batch, partition=S) evaluates the split partials with that S and merges them ([FvP] eq. (4)).
+
+    The partials are watched on their way through the module: step() must ask
+    for partitions of exactly S tokens over the appended caches (finite, since
+    the pre-append pools hold NaN in the new slots), and the merged rows equal
+    the single-pass rows for S = B (one block per partition) and S = 512 (one
+    partition per sequence).
+    """
+    b = small_decode(seed=121, lens=(1, 9, 16, 31, 64, 77))
+    ref, *_ = P.step(b)
+    real = P.splitkv_partials
+    for S in (b.block_size, 512):
+        seen = []
+
+        def spy(q, k_cache, v_cache, block_tables, context_lens, scale, partition, num_parts=None):
+            r = real(q, k_cache, v_cache, block_tables, context_lens, scale, partition, num_parts)
+            seen.append((partition, bool(np.isfinite(r[0]).all())))
+            return r
+
+        P.splitkv_partials = spy
+        try:
+            out, *_ = P.step(b, partition=S)
+        finally:
+            P.splitkv_partials = real
+        assert seen == [(S, True)], seen
+        np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
 ALL_PINS = [
     pin_uniform_scores_mean_of_v, pin_dominant_key, pin_single_token, pin_block_permutation,
     pin_shared_vs_private, pin_eq4_block_sums, pin_partials_closed_form, pin_merge_empty,
     pin_torch_sdpa, pin_brute_force, pin_prefill_rows_are_truncated_decodes,
-    pin_page_example_slots, pin_cache_write, pin_copy_blocks,
+    pin_page_example_slots, pin_cache_write, pin_copy_blocks, pin_step_appends_then_attends,
+    pin_step_partition_branch,
 ]

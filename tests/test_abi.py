@@ -65,6 +65,48 @@ def test_num_partitions(lib):
     assert f(10, 0) == 0
 
 
+def test_splitkv_workspace_bytes(lib):
+    """The section 8(b) workspace query: three fp32 parts, each rounded up to 256 bytes; 0 when invalid."""
+    f = lib.pa_splitkv_workspace_bytes
+    f.restype = ctypes.c_size_t
+    r256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    # 100k split-KV shape: 4 x 32 rows, 196 partitions of 512 tokens, D = 128
+    cells = 4 * 32 * 196
+    assert f(4, 32, 128, 100000, 512) == r256(cells * 128 * 4) + 2 * r256(cells * 4)
+    # one partition per row even for an empty context; a 1-cell part still takes 256 bytes
+    assert f(1, 1, 64, 0, 512) == r256(64 * 4) + 2 * 256
+    assert f(3, 5, 64, 513, 512) == r256(3 * 5 * 2 * 64 * 4) + 2 * r256(3 * 5 * 2 * 4)
+    assert f(0, 32, 128, 4096, 512) == 0
+    for bad in [(-1, 32, 128, 4096, 512), (4, 0, 128, 4096, 512), (4, 32, 0, 4096, 512), (4, 32, 128, -5, 512),
+                (4, 32, 128, 4096, 0)]:
+        assert f(*bad) == 0, bad
+    # sizes that do not fit in size_t report 0 rather than a wrapped value
+    assert f(2**31 - 1, 2**31 - 1, 2**31 - 1, 2**31 - 1, 16) == 0
+
+
+def _noalloc_args(**kw):
+    fake = ctypes.c_void_p(256)  # never dereferenced: every case below is refused on the host
+    a = dict(out=fake, q=fake, k=fake, v=fake, bt=fake, mb=4, lens=fake, N=2, Hq=8, Hkv=2, D=128, B=16, P=10,
+             part=512, np=4, scale=ctypes.c_float(0.1), dt=1, stream=None)
+    a.update(kw)
+    return list(a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    # rows * partitions * (D + 2) * 4 bytes far beyond the 16 MiB array
+    (dict(np=100_000), -5),
+    # a product that would wrap 64 bits if formed naively: 65535 x 2^31-1 rows ...
+    (dict(N=65535, Hq=2**31 - 1, Hkv=2**31 - 1, np=2**30), -5),
+    (dict(N=65535, Hq=2**31 - 1, Hkv=2**31 - 1, np=2**30 + 1), -2),  # ... or a partition count past 2^30
+    (dict(N=1, Hq=8, np=2**30 + 1), -2),
+    (dict(N=65536), -2),
+    (dict(part=24), -5), (dict(np=0), -5), (dict(out=None), -1),
+])
+def test_noalloc_rejects_oversized_or_absurd_shapes_on_host(lib, kw, code):
+    """pa_decode_splitkv_noalloc refuses before any CUDA call (these run without a GPU)."""
+    assert lib.pa_decode_splitkv_noalloc(*_noalloc_args(**kw)) == code
+
+
 def _decode_args(**kw):
     fake = ctypes.c_void_p(16)  # never dereferenced: validation fails first
     a = dict(out=fake, q=fake, k=fake, v=fake, bt=fake, mb=4, lens=fake, N=2, Hq=8, Hkv=2, D=128, B=16, P=10,
@@ -160,6 +202,10 @@ int main(void) {
   if (strcmp(pa_status_string(PA_OK), "PA_OK") != 0) fails++;
   if (pa_version() < 100) fails++;
   if (pa_splitkv_num_partitions(100000, 512) != 196) fails++;
+  /* one workspace for part_o [4,32,196,128], part_m and part_l [4,32,196], each rounded to 256 B */
+  if (pa_splitkv_workspace_bytes(4, 32, 128, 100000, 512) != (size_t)(4 * 32 * 196 * 128 * 4 + 2 * 100352))
+    fails++;
+  if (pa_splitkv_workspace_bytes(4, 0, 128, 100000, 512) != 0) fails++;
   /* host-side checks run before any device work */
   char fake[256];
   if (pa_decode(fake, fake, fake, fake, (const int32_t*)fake, 4, (const int32_t*)fake, 2, 8, 2, 96, 16, 10,

@@ -4,7 +4,9 @@ Each mutant swaps one oracle function for a copy with one plausible slip in
 it: a dropped scale, a wrong KV head, pages in the wrong order, an off-by-one
 causal limit, a sign error, a merge that forgets a weight, a slot formula with
 block and offset swapped, a cache write one row off, a merge in the wrong log
-base, a slot that skips the block table, K and V swapped. The real oracle passes
+base, a slot that skips the block table, K and V swapped, a step that attends
+before its append, ignores the split-KV partition or appends one position
+late. The real oracle passes
 every pin (tests/test_oracle.py); a pin set that let any of these through would
 not be pinning the oracle.
 """
@@ -134,7 +136,45 @@ def cache_write_swaps_kv(k_new, v_new, k_cache, v_cache, slots):
     return _orig_rc(v_new, k_new, k_cache, v_cache, slots)
 
 
+def step_attends_before_append(batch, partition=None):
+    """Appends, but attends over the caches as they were before the append."""
+    slots = P.slot_mapping(batch.block_tables, batch.new_seq, batch.new_pos, batch.block_size)
+    kc, vc = P.reshape_and_cache(batch.k_new, batch.v_new, batch.k_cache, batch.v_cache, slots)
+    if partition is not None:
+        o, m, l = P.splitkv_partials(batch.q, batch.k_cache, batch.v_cache, batch.block_tables, batch.context_lens,
+                                     batch.scale, partition)
+        return P.merge(o, m, l), kc, vc, slots
+    out = P.attention(batch.q, batch.k_cache, batch.v_cache, batch.block_tables, batch.context_lens, batch.scale)
+    return out, kc, vc, slots
+
+
+def step_ignores_partition(batch, partition=None):
+    """Drops the split-KV branch: always the single pass."""
+    return _orig_step(batch)
+
+
+def step_partition_pre_append(batch, partition=None):
+    """Split branch only: partials over the pre-append caches."""
+    if partition is None:
+        return _orig_step(batch)
+    return step_attends_before_append(batch, partition)
+
+
+def step_appends_next_position(batch, partition=None):
+    """Writes each new token one position later than its own."""
+    slots = P.slot_mapping(batch.block_tables, batch.new_seq, batch.new_pos + 1, batch.block_size)
+    kc, vc = P.reshape_and_cache(batch.k_new, batch.v_new, batch.k_cache, batch.v_cache, slots)
+    out = P.attention(batch.q, kc, vc, batch.block_tables, batch.context_lens, batch.scale)
+    return out, kc, vc, slots
+
+
+_orig_step = P.step
+
 MUTANTS = {
+    "step_attends_before_append": ("step", step_attends_before_append),
+    "step_ignores_partition": ("step", step_ignores_partition),
+    "step_partition_pre_append": ("step", step_partition_pre_append),
+    "step_appends_next_position": ("step", step_appends_next_position),
     "merge_exp2_units": ("merge", merge_exp2_units),
     "slots_ignore_table": ("slot_mapping", slots_ignore_table),
     "cache_write_swaps_kv": ("reshape_and_cache", cache_write_swaps_kv),
