@@ -64,7 +64,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llama_decode", choices=list(WORKLOAD_DESC))
+    ap.add_argument("--workload", default="llama_decode", choices=list(WORKLOAD_DESC) + ["block_swap"])
     ap.add_argument("--block-size", type=int, default=16)
     ap.add_argument("--partition", default="auto")
     ap.add_argument("--no-e2e", action="store_true")
@@ -718,6 +718,96 @@ def measure(name, block_size, partition_arg, K, W, rank, world, sampler, do_e2e=
     return res
 
 
+def measure_block_swap(K, W, rank, world, runs=64, run_blocks=32):
+    """Block copies of the Llama-shaped pool (8 KV heads x 16 tokens x 128 dims, fp16: 64 KiB of K+V per
+    block): swap-out to and swap-in from a pinned host pool through pa_copy_blocks (the kernel reads or
+    writes host memory directly), the same bytes as one cudaMemcpyAsync per contiguous run of blocks, and
+    a device-side copy-on-write of as many blocks. Every figure is bytes moved / CUDA-event time."""
+    import torch
+
+    import paged_kv_cache_475_b200 as pa
+
+    Hkv, B, D = 8, 16, 128
+    n = runs * run_blocks
+    P_dev = 4 * n
+    g = torch.Generator().manual_seed(5 + 100 * rank)
+    kd = torch.randn((P_dev, Hkv, B, D), generator=g).to(torch.float16).cuda()
+    vd = torch.randn((P_dev, Hkv, B, D), generator=g).to(torch.float16).cuda()
+    kh = torch.empty((n, Hkv, B, D), dtype=torch.float16).pin_memory()
+    vh = torch.empty((n, Hkv, B, D), dtype=torch.float16).pin_memory()
+    starts = (torch.randperm(P_dev // run_blocks, generator=g)[:runs] * run_blocks).tolist()
+    dev_ids = torch.tensor([s0 + j for s0 in starts for j in range(run_blocks)], dtype=torch.int32)
+    host_ids = torch.arange(n, dtype=torch.int32)
+    dev_ids_g, host_ids_g = dev_ids.cuda(), host_ids.cuda()
+    block_bytes = 2 * Hkv * B * D * 2
+    moved = n * block_bytes
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(W):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1), world) / K
+
+    def out_kernel():
+        pa.pa_copy_blocks(kh, vh, kd, vd, dev_ids_g, host_ids_g)
+
+    def in_kernel():
+        pa.pa_copy_blocks(kd, vd, kh, vh, host_ids_g, dev_ids_g)
+
+    def out_memcpy():
+        for r, s0 in enumerate(starts):
+            h0 = r * run_blocks
+            kh[h0:h0 + run_blocks].copy_(kd[s0:s0 + run_blocks], non_blocking=True)
+            vh[h0:h0 + run_blocks].copy_(vd[s0:s0 + run_blocks], non_blocking=True)
+
+    def in_memcpy():
+        for r, s0 in enumerate(starts):
+            h0 = r * run_blocks
+            kd[s0:s0 + run_blocks].copy_(kh[h0:h0 + run_blocks], non_blocking=True)
+            vd[s0:s0 + run_blocks].copy_(vh[h0:h0 + run_blocks], non_blocking=True)
+
+    kd_one = kd[:n]
+    cow_src = dev_ids_g
+    cow_dst = torch.tensor([(int(i) + 2 * n) % P_dev for i in dev_ids], dtype=torch.int32).cuda()
+
+    def cow_kernel():
+        pa.pa_copy_blocks(kd, vd, kd, vd, cow_src, cow_dst)
+
+    res = {}
+    for name, fn in (("swap_out_kernel", out_kernel), ("swap_in_kernel", in_kernel),
+                     ("swap_out_memcpy_per_run", out_memcpy), ("swap_in_memcpy_per_run", in_memcpy)):
+        ms = timed(fn)
+        res[name] = {"ms": ms, "GB/s": moved / (ms / 1e3) / 1e9}
+    ms = timed(lambda: kh.copy_(kd_one, non_blocking=True))
+    res["one_memcpy_d2h_half_bytes"] = {"ms": ms, "GB/s": moved / 2 / (ms / 1e3) / 1e9}
+    ms = timed(lambda: kd_one.copy_(kh, non_blocking=True))
+    res["one_memcpy_h2d_half_bytes"] = {"ms": ms, "GB/s": moved / 2 / (ms / 1e3) / 1e9}
+    ms = timed(cow_kernel)
+    hbm_peak, _, peak_src = measured_peaks()
+    res["copy_on_write_device"] = {"ms": ms, "GB/s": 2 * moved / (ms / 1e3) / 1e9,
+                                   "hbm_frac": 2 * moved / (ms / 1e3) / 1e9 / hbm_peak,
+                                   "bytes": "read + write of every copied block"}
+    flags = pa.pa_read_error_flags(clear=True)
+    # the swapped-out blocks really are the device blocks, bit for bit
+    out_kernel()
+    torch.cuda.synchronize()
+    ok = bool(torch.equal(kh.view(torch.int16), kd[dev_ids.long()].cpu().view(torch.int16)))
+    res.update({"blocks": n, "runs": runs, "blocks_per_run": run_blocks, "bytes_per_direction": moved,
+                "block_bytes": block_bytes, "bit_exact_roundtrip": ok, "device_error_flags": flags,
+                "peak_source": peak_src,
+                "pool": "Llama-shaped fp16 pool [P, 8, 16, 128] for K and for V; host pool pinned"})
+    del kd, vd, kh, vh
+    torch.cuda.empty_cache()
+    return res
+
+
 EXTRA_WORKLOADS = ("long_context", "chat_trace", "prefill_chunk")
 SWEEP_BLOCK_SIZES = (8, 16, 32, 64, 128)
 
@@ -726,6 +816,11 @@ def run_ours(args):
     import torch
 
     world, rank, local = dist_init(args)
+    if args.workload == "block_swap":  # the block copies alone (swap out / in, copy-on-write)
+        r = measure_block_swap(args.steps, args.warmup, rank, world)
+        if rank == 0:
+            print(json.dumps({"workload": "block_swap", **r}))
+        return
     sampler = ClockSampler(local)
     sampler.start()
     K, W = args.steps, args.warmup
@@ -738,6 +833,7 @@ def run_ours(args):
         for name in EXTRA_WORKLOADS:
             extras[name] = measure(name, 16, "auto", K, W, rank, world, sampler, do_e2e=not args.no_e2e,
                                    sustain_s=args.sustain_seconds)
+        swap = measure_block_swap(K, W, rank, world)
         for B in SWEEP_BLOCK_SIZES:  # the pages' block-size question, on the chat trace (cascade)
             r = measure("chat_trace", B, "auto", K, W, rank, world, sampler, do_e2e=False, sustain_s=0.0)
             sweep.append({"block_size": B, "value": r["value"], "unit": r["unit"], "ms_per_step": r["ms_per_step"],
@@ -779,6 +875,7 @@ def run_ours(args):
                 r.pop("warmup", None)
                 line["workloads"][name] = r
             line["workloads"]["chat_trace"]["block_size_sweep"] = sweep
+            line["workloads"]["block_swap"] = swap
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist

@@ -232,14 +232,18 @@ PA_API int pa_decode_splitkv(float* part_o, float* part_m, float* part_l, const 
  * of pa_decode_append), computed as a cascade:
  *   1) the group's G*group_size query rows of each KV head attend to the shared
  *      prefix pages once, as a dense tile on the tensor cores (read through
- *      block_tables row 0); the prefix keys are cut into S = 4, 2 or 1 equal
- *      ranges (multiples of 128 keys, S + 1 <= num_partitions), one partial
- *      slot each;
+ *      block_tables row 0); the prefix keys form S equal ranges, one partial
+ *      slot each: S = 1, or 2 or 4 when a range would otherwise exceed 4096
+ *      keys (ranges are multiples of 128 keys, S + 1 <= num_partitions);
  *   2) one pass per (sequence, KV head) over the sequence's own tokens: group
  *      members from token prefix_len on, written as partials into slot S; all
  *      other sequences whole, written straight to `out`; the newest token's
  *      row written first if given;
  *   3) the group's rows: log-sum-exp merge of slots 0..S.
+ * Passes 1 and 2 touch disjoint data, so pass 1 runs on a stream the library
+ * keeps per device (created on the first call with that device current, and
+ * again after a device reset), forked from and joined back to `stream` by
+ * events before pass 3; stream capture records the fork and the join.
  * part_o/part_m/part_l: caller workspace [N, Hq, num_partitions(, D)] fp32,
  * num_partitions >= 2 (5 lets S reach 4). Needs prefix_len a positive
  * multiple of 16 and of B, every group member with L_b > prefix_len (else
@@ -353,6 +357,22 @@ PA_API const char* pa_last_cuda_error(void);
 
 /* Human-readable name of a pa_status value. */
 PA_API const char* pa_status_string(int status);
+
+/*
+ * Timeline tracing, for builds made with -DPA_TRACE=1 (python
+ * paged_kv_cache_475_b200/build.py --trace); every other build returns
+ * PA_ERR_UNSUPPORTED from both calls. A traced decode kernel writes one
+ * record per CTA (linear CTA index, at most 65536) into a device array:
+ *   struct { uint64 t_start, t_first, t_end;   global timer, ns: entry, first
+ *                                               tile landed (warp 0), exit
+ *            int32 smid, seq, kv_head, part, tokens, kind; }  (48 bytes)
+ * pa_trace_clear zeroes the array (synchronises); pa_trace_read synchronises
+ * and copies max_records records to host memory. The records of the last
+ * traced launch overwrite those of earlier ones. Not part of the attention
+ * path: the pages have no counterpart; it measures where a kernel's time goes.
+ */
+PA_API int pa_trace_clear(void);
+PA_API int pa_trace_read(void* host_records, int max_records);
 
 /* Library ABI version (major * 100 + minor): 101 adds pa_splitkv_workspace_bytes. */
 PA_API int pa_version(void);

@@ -58,6 +58,8 @@ _SIGS = {
     "pa_status_string": [_i],
     "pa_last_cuda_error": [],
     "pa_version": [],
+    "pa_trace_clear": [],
+    "pa_trace_read": [_vp, _i],
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -334,6 +336,22 @@ def pa_decode_splitkv_noalloc(out, q, k_cache, v_cache, block_tables, context_le
 
 def pa_noalloc_scratch_bytes() -> int:
     return _lib.pa_noalloc_scratch_bytes()
+
+
+def trace_clear() -> None:
+    """Zero the timeline records (builds with PA_TRACE=1 only; see include/pa.h)."""
+    _check(_lib.pa_trace_clear(), "pa_trace_clear")
+
+
+def trace_read(max_records: int = 1 << 16):
+    """Timeline records of the last traced launch as a numpy structured array (PA_TRACE=1 builds only)."""
+    import numpy as np
+
+    dt = np.dtype([("t_start", "<u8"), ("t_first", "<u8"), ("t_end", "<u8"), ("smid", "<i4"), ("seq", "<i4"),
+                   ("kv_head", "<i4"), ("part", "<i4"), ("tokens", "<i4"), ("kind", "<i4")])
+    buf = np.zeros(max_records, dtype=dt)
+    _check(_lib.pa_trace_read(ctypes.c_void_p(buf.ctypes.data), int(max_records)), "pa_trace_read")
+    return buf
 
 
 def pa_read_error_flags(clear: bool = True) -> int:

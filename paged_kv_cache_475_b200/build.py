@@ -39,8 +39,20 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
+def _flags_file(lib: str) -> str:
+    return lib + ".defines"
+
+
+def _stale(defines=()) -> bool:
     if not os.path.exists(LIB):
+        return True
+    # a library built with other -D macros (e.g. a --trace build) is rebuilt
+    try:
+        with open(_flags_file(LIB)) as f:
+            built_with = f.read().split()
+    except OSError:
+        built_with = []
+    if sorted(built_with) != sorted(defines):
         return True
     t = os.path.getmtime(LIB)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [HEADER]
@@ -52,7 +64,7 @@ def build(force: bool = False, verbose: bool = False, defines=(), lib: str = LIB
 
     defines: extra -D macros (tuning variants), written to `lib` with objects in `objdir`.
     """
-    if not force and os.path.abspath(lib) == LIB and not _stale():
+    if not force and os.path.abspath(lib) == LIB and not _stale(tuple(defines)):
         return LIB
     os.makedirs(objdir, exist_ok=True)
     cc = nvcc()
@@ -82,6 +94,8 @@ def build(force: bool = False, verbose: bool = False, defines=(), lib: str = LIB
     if r.returncode:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, lib)
+    with open(_flags_file(lib), "w") as f:
+        f.write(" ".join(defines))
     return lib
 
 
@@ -89,5 +103,7 @@ if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--trace", action="store_true",
+                    help="build with per-CTA timeline records (PA_TRACE=1; pa_trace_read), off by default")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force or a.trace, verbose=a.verbose, defines=("PA_TRACE=1",) if a.trace else ()))

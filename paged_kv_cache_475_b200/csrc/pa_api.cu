@@ -64,6 +64,46 @@ int record_cuda_error(cudaError_t e, const char* where) {
 
 }  // namespace pa
 
+namespace pa {
+#if PA_TRACE
+__device__ TraceRecord g_trace[kTraceMax];
+#endif
+TraceRecord* trace_buffer() {
+#if PA_TRACE
+  void* p = nullptr;
+  return cudaGetSymbolAddress(&p, g_trace) == cudaSuccess ? static_cast<TraceRecord*>(p) : nullptr;
+#else
+  return nullptr;
+#endif
+}
+}  // namespace pa
+
+extern "C" PA_API int pa_trace_read(void* host_records, int max_records) {
+#if PA_TRACE
+  if (!host_records || max_records <= 0) return PA_ERR_NULL;
+  const int n = max_records < pa::kTraceMax ? max_records : pa::kTraceMax;
+  if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
+  const cudaError_t e = cudaMemcpyFromSymbol(host_records, pa::g_trace, sizeof(pa::TraceRecord) * n);
+  if (e != cudaSuccess) return pa::record_cuda_error(e, "trace: copy the records");
+  return PA_OK;
+#else
+  (void)host_records;
+  (void)max_records;
+  return PA_ERR_UNSUPPORTED;
+#endif
+}
+
+extern "C" PA_API int pa_trace_clear(void) {
+#if PA_TRACE
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, pa::g_trace) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaMemset(p, 0, sizeof(pa::TraceRecord) * pa::kTraceMax) != cudaSuccess) return PA_ERR_CUDA;
+  return cudaDeviceSynchronize() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+#else
+  return PA_ERR_UNSUPPORTED;
+#endif
+}
+
 extern "C" PA_API const char* pa_last_cuda_error(void) { return pa::g_last_error; }
 
 extern "C" PA_API int pa_read_error_flags(uint32_t* host_flags, int clear) {

@@ -236,6 +236,36 @@ __device__ inline void set_error(unsigned int* err, unsigned int bit) {
   if (err) atomicOr(err, bit);
 }
 
+// ---------------------------------------------------------------------------
+// Timeline tracing (builds with -DPA_TRACE=1 only; off by default). A traced
+// kernel stamps, per CTA, the global timer at entry, when its first tile has
+// landed, and at exit, with the SM it ran on and the work it did; the records
+// go to a fixed device array that pa_trace_read copies out.
+// ---------------------------------------------------------------------------
+#ifndef PA_TRACE
+#define PA_TRACE 0
+#endif
+struct TraceRecord {
+  unsigned long long t_start, t_first, t_end;  // %globaltimer, ns
+  int smid, seq, kv_head, part, tokens, kind;
+};
+constexpr int kTraceMax = 1 << 16;
+// Device address of the record array (lives in pa_api.cu; every .cu is its own
+// device module, so kernels get the address as a parameter); null unless PA_TRACE.
+TraceRecord* trace_buffer();
+#if PA_TRACE
+__device__ inline unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ inline int sm_id() {
+  int s;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(s));
+  return s;
+}
+#endif
+
 // Packed fp32 FMA (sm_100): {a.x*b.x + c.x, a.y*b.y + c.y} in one instruction.
 __device__ inline float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 

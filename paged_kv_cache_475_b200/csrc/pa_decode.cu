@@ -83,32 +83,45 @@ struct DecodeParams {
   int cascade_prefix;
   int cascade_group;
   int cascade_slot;
+  TraceRecord* trace;        // timeline records (PA_TRACE builds), else null
 };
 
-// Sequence whose context is the r-th longest (ties by index). CTAs are
-// dispatched in z order, so the longest contexts start first and short ones
-// fill the tail (greedy longest-processing-time scheduling). The lengths are
-// staged in shared memory (`work`, n ints) with one coalesced load, then each
-// thread ranks its own sequences against them: O(N^2 / threads) shared-memory
-// compares per CTA, used for small batches only.
+// Sequence whose work is the r-th largest (ties by index). CTAs are dispatched
+// in z order, so the longest contexts start first and short ones fill the
+// tail (greedy longest-processing-time scheduling). The CTA stages one 64-bit
+// key per sequence in shared memory (`keys`, room for the next power of two
+// >= n), high word the work + 2^31, low word the complement of the index, and
+// sorts them in descending order with a bitonic network: log2(n)(log2(n)+1)/2
+// compare-exchange rounds, n/2 pairs each, spread over the CTA's threads.
 // Work of sequence j is its length minus `skip` tokens when j < group.
-__device__ inline int longest_first_seq(const int32_t* lens, int n, int r, int* slot, int* work,
-                                        int group = 0, int skip = 0) {
-  for (int j = threadIdx.x; j < n; j += blockDim.x) work[j] = lens[j] - (j < group ? skip : 0);
-  if (threadIdx.x == 0) *slot = r;
-  __syncthreads();
-  for (int j = threadIdx.x; j < n; j += blockDim.x) {
-    const int Lj = work[j];
-    int rank = 0;
-#pragma unroll 8
-    for (int i = 0; i < n; ++i) {
-      const int Li = work[i];
-      rank += (Li > Lj) || (Li == Lj && i < j);
+__device__ inline int longest_first_seq(const int32_t* lens, int n, int r, unsigned long long* keys, int group = 0,
+                                        int skip = 0) {
+  int n2 = 1;
+  while (n2 < n) n2 <<= 1;
+  for (int j = threadIdx.x; j < n2; j += blockDim.x) {
+    unsigned long long k = 0;  // padding sorts after every real key
+    if (j < n) {
+      const int w = lens[j] - (j < group ? skip : 0);
+      k = (static_cast<unsigned long long>(static_cast<unsigned>(w) + 0x80000000u) << 32) |
+          static_cast<unsigned long long>(0xffffffffu - static_cast<unsigned>(j));
     }
-    if (rank == r) *slot = j;
+    keys[j] = k;
   }
   __syncthreads();
-  const int b = *slot;
+  for (int size = 2; size <= n2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = threadIdx.x; t < (n2 >> 1); t += blockDim.x) {
+        const int i = 2 * stride * (t / stride) + (t % stride);  // lower index of the pair
+        const unsigned long long a = keys[i], c = keys[i + stride];
+        if ((a < c) == ((i & size) == 0)) {  // descending blocks put the larger key first
+          keys[i] = c;
+          keys[i + stride] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const int b = static_cast<int>(0xffffffffu - static_cast<unsigned>(keys[r] & 0xffffffffull));
   __syncthreads();  // the staging area is the copy ring, which the caller fills next
   return b;
 }
@@ -208,12 +221,11 @@ struct DecodeSmem {
   static constexpr int kTotal = kValidOff + NW * STAGES * 4 + 16;
 };
 
-#ifndef PA_DECODE_MINB
-#define PA_DECODE_MINB 1
-#endif
-
+// No minimum-blocks bound: the fp16 / bf16 kernels at D = 128 fit three CTAs
+// per SM (167 registers, 67 KB) without one, and capping the registers at 170
+// to force it made the compiler trade ILP for registers (2.5% slower).
 template <typename T, int D, int G, int NW, int STAGES>
-__global__ void __launch_bounds__(NW * 32, PA_DECODE_MINB)
+__global__ void __launch_bounds__(NW * 32, 1)
 decode_kernel(const DecodeParams p) {
   using S = DecodeShape<T, D, G>;
   using M = DecodeSmem<T, D, G, NW, STAGES>;
@@ -224,6 +236,10 @@ decode_kernel(const DecodeParams p) {
   const int part = blockIdx.x;
   const int kvh = blockIdx.y;
   const bool split = p.partition > 0;
+#if PA_TRACE
+  const unsigned long long tr_start = global_ns();
+  unsigned long long tr_first = 0;
+#endif
   // A shared prefix's partition was computed once for its whole group; a
   // group member must reach past the prefix (its newest token is its own).
   if (split && part == 0 && static_cast<int>(blockIdx.z) < p.skip_part0_seqs) {
@@ -232,8 +248,8 @@ decode_kernel(const DecodeParams p) {
   }
   const int b = p.longest_first
                     ? longest_first_seq(p.context_lens, p.num_seqs, blockIdx.z,
-                                        reinterpret_cast<int*>(smem + M::kValidOff + NW * STAGES * 4),
-                                        reinterpret_cast<int*>(smem), p.cascade_group, p.cascade_prefix)
+                                        reinterpret_cast<unsigned long long*>(smem), p.cascade_group,
+                                        p.cascade_prefix)
                     : static_cast<int>(blockIdx.z);
   const bool cascade_member = p.cascade_prefix > 0 && b < p.cascade_group;
   if (cascade_member && threadIdx.x == 0 && kvh == 0 && p.context_lens[b] <= p.cascade_prefix)
@@ -415,6 +431,9 @@ decode_kernel(const DecodeParams p) {
       aborted = true;
       break;
     }
+#if PA_TRACE
+    if (k == 0 && warp == 0) tr_first = global_ns();
+#endif
     const int nvalid = stage_valid[s];
     const unsigned char* ktile = ring + s * M::kStageBytes;
     const unsigned char* vtile = ktile + S::kTileBytes;
@@ -600,6 +619,14 @@ decode_kernel(const DecodeParams p) {
       out[d] = Elem<T>::from_f(l > 0.f ? o / l : 0.f);
     }
   }
+#if PA_TRACE
+  if (threadIdx.x == 0) {
+    const long long idx = blockIdx.x + static_cast<long long>(gridDim.x) * (blockIdx.y + static_cast<long long>(gridDim.y) * blockIdx.z);
+    if (p.trace != nullptr && idx < kTraceMax)
+      p.trace[idx] = TraceRecord{tr_start, tr_first, global_ns(), sm_id(), b, kvh, part, t_end - t_begin,
+                                 split ? 1 : (cascade_member ? 2 : 0)};
+  }
+#endif
 }
 
 // ---------------------------------------------------------------------------
@@ -703,7 +730,7 @@ merge_kernel(T* __restrict__ out, const float* __restrict__ part_o, const float*
 #define PA_DECODE_STAGES 2
 #endif
 #ifndef PA_DECODE_LPT_MAX_SEQS
-#define PA_DECODE_LPT_MAX_SEQS 256
+#define PA_DECODE_LPT_MAX_SEQS 512  // 512 x 8-byte keys fit the smallest copy ring (32 KB)
 #endif
 constexpr int kDecodeWarps = PA_DECODE_WARPS;
 constexpr int kDecodeStages = PA_DECODE_STAGES;
@@ -719,8 +746,11 @@ int launch_decode(const DecodeParams& prm, int grid_x, cudaStream_t stream) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !attr_done[dev].valid()) {
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, M::kTotal);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, M::kTotal);
     if (e != cudaSuccess) return record_cuda_error(e, "decode: set max dynamic shared memory");
+    // all of the SM's unified L1/shared memory as shared memory, so that three CTAs fit
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return record_cuda_error(e, "decode: set the shared memory carveout");
     if (dev >= 0 && dev < 64) attr_done[dev].set(true);
   }
   dim3 grid(grid_x, prm.num_kv_heads, prm.num_seqs);
@@ -750,6 +780,7 @@ int run_decode(DecodeParams prm, int D, float scale, pa_dtype dt, int grid_x, cu
   const int G = prm.num_q_heads / prm.num_kv_heads;
   prm.q_scale = scale * kLog2e;
   prm.err = device_error_word();
+  prm.trace = trace_buffer();
   switch (dt) {
     case PA_F32: return dispatch_dim<float>(prm, D, G, grid_x, s);
     case PA_F16: return dispatch_dim<__half>(prm, D, G, grid_x, s);
@@ -970,6 +1001,42 @@ int launch_merge_any(void* out, const float* po, const float* pm, const float* p
 }
 }  // namespace pa
 
+namespace pa {
+namespace {
+// A side stream per device on which pa_decode_shared_prefix runs the shared
+// prompt's pass concurrently with the suffix pass on the caller's stream
+// (fork and join by events, which stream capture also records). Created on
+// first use with that device current, and again after a device reset.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  uint64_t ctx = 0;
+};
+SideStream g_side[64];
+std::mutex g_side_mu;  // held from the fork to the join, so concurrent callers never share an event record
+
+int side_stream_locked(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record_cuda_error(e, "shared prefix: current device");
+  if (dev < 0 || dev >= 64) return PA_ERR_UNSUPPORTED;
+  SideStream& ss = g_side[dev];
+  const uint64_t now = current_context_id();
+  if (ss.stream == nullptr || now == 0 || now != ss.ctx) {
+    SideStream fresh;
+    e = cudaStreamCreateWithFlags(&fresh.stream, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&fresh.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&fresh.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) return record_cuda_error(e, "shared prefix: create the side stream");
+    fresh.ctx = current_context_id();
+    ss = fresh;  // handles of a context that a reset destroyed are gone with it
+  }
+  *out = &ss;
+  return PA_OK;
+}
+}  // namespace
+}  // namespace pa
+
 extern "C" PA_API int pa_decode_shared_prefix(void* out, const void* q, const void* k_new, const void* v_new,
                                               void* k_cache, void* v_cache, const int32_t* block_tables,
                                               int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
@@ -989,18 +1056,33 @@ extern "C" PA_API int pa_decode_shared_prefix(void* out, const void* q, const vo
   if (num_partitions < 2) return PA_ERR_WORKSPACE;
   if (num_seqs > 65535) return PA_ERR_SHAPE;
   cudaStream_t s = (cudaStream_t)stream;
-  // Split the prefix keys over up to 4 CTA rows (each a multiple of 128 keys)
-  // so the prefix pass fills the GPU; its slots are 0..splits-1, the
-  // suffix pass writes slot `splits`.
+  // The prefix pass runs beside the suffix pass, one CTA per SM, so it should
+  // hold few SMs: its keys are cut into more than one range (up to 4, each a
+  // multiple of 128 keys) only when a range would exceed 4096 keys. Its slots
+  // are 0..splits-1; the suffix pass writes slot `splits`.
   int splits = 1;
-  for (int c : {4, 2})
-    if (splits == 1 && prefix_len % (128 * c) == 0 && c + 1 <= num_partitions) splits = c;
-  // 1) the shared prefix, once for the whole group, on the tensor cores
+  for (int c : {2, 4})
+    if (prefix_len / splits > 4096 && prefix_len % (128 * c) == 0 && c + 1 <= num_partitions) splits = c;
+  // 1) the shared prefix, once for the whole group, on the tensor cores. It
+  //    reads no row that pass 2 writes (the appended rows lie past the prefix)
+  //    and writes other partial slots, so it runs on a side stream while pass
+  //    2 runs on the caller's stream; the merge waits for both.
+  std::unique_lock<std::mutex> side_lock(g_side_mu, std::defer_lock);
+  SideStream* side = nullptr;
+  int prefix_st = PA_OK;
   if (group_size > 0) {
-    PrefixPartials pp{prefix_len, part_o, part_m, part_l, num_partitions, splits};
-    st = prefill_tcgen05(nullptr, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, 1, group_size,
-                         num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, dtype, s, &pp);
+    side_lock.lock();
+    st = side_stream_locked(&side);
     if (st != PA_OK) return st;
+    cudaError_t e = cudaEventRecord(side->fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
+    if (e != cudaSuccess) return record_cuda_error(e, "shared prefix: fork to the side stream");
+    PrefixPartials pp{prefix_len, part_o, part_m, part_l, num_partitions, splits};
+    prefix_st = prefill_tcgen05(nullptr, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, 1,
+                                group_size, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, dtype,
+                                side->stream, &pp);
+    e = cudaEventRecord(side->join, side->stream);
+    if (e != cudaSuccess) return record_cuda_error(e, "shared prefix: record the join");
   }
   // 2) every sequence's own tokens in one pass per (sequence, KV head): group
   //    members from prefix_len on (partials), the others whole (final rows);
@@ -1030,7 +1112,12 @@ extern "C" PA_API int pa_decode_shared_prefix(void* out, const void* q, const vo
   prm.cascade_slot = splits;
   prm.longest_first = num_seqs > 1 && num_seqs <= PA_DECODE_LPT_MAX_SEQS;
   st = run_decode(prm, head_dim, scale, dtype, 1, s);
-  if (st != PA_OK || group_size == 0) return st;
+  if (group_size == 0) return st;
+  const cudaError_t e = cudaStreamWaitEvent(s, side->join, 0);  // join, whatever happened above
+  side_lock.unlock();
+  if (e != cudaSuccess) return record_cuda_error(e, "shared prefix: join the side stream");
+  if (prefix_st != PA_OK) return prefix_st;
+  if (st != PA_OK) return st;
   // 3) the group's rows: log-sum-exp merge of the prefix slots and the suffix slot
   return launch_merge_any(out, part_o, part_m, part_l, context_lens, group_size * num_q_heads, num_q_heads,
                           head_dim, -(splits + 1), num_partitions, dtype, s);

@@ -1,0 +1,89 @@
+"""Per-CTA timeline of one decode step (needs a build made with `build.py --trace`).
+
+python -m paged_kv_cache_475_b200.trace --workload llama_decode|chat_trace|long_context [--out t.npz]
+
+Runs a few warm-up steps of the workload (the same step bench.py times), then
+one step with the timeline records cleared before it, and prints where the
+decode kernel's time goes: how long a CTA waits from entry until its first
+tile has landed, how many CTAs each SM runs over time, and how the kernel
+ends (the tail, when SMs run out of CTAs). The records are written to --out
+as a numpy archive for further study.
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def summarize(rec, num_sms=148, bins=20):
+    rec = rec[rec["t_start"] > 0]
+    t0 = rec["t_start"].min()
+    start = (rec["t_start"] - t0) / 1e3
+    first = np.where(rec["t_first"] > 0, (rec["t_first"] - t0) / 1e3, np.nan)
+    end = (rec["t_end"] - t0) / 1e3
+    span = end.max()
+    out = {"ctas": int(len(rec)), "span_us": float(span),
+           "first_tile_after_entry_us": {q: float(np.nanpercentile(first - start, p))
+                                         for q, p in (("p10", 10), ("median", 50), ("p90", 90))},
+           "cta_life_us": {q: float(np.percentile(end - start, p)) for q, p in (("p10", 10), ("median", 50),
+                                                                                 ("p90", 90), ("max", 100))},
+           "last_cta_start_us": float(start.max())}
+    # CTAs resident per SM over time, and the share of CTA-time spent before the first tile
+    edges = np.linspace(0, span, bins + 1)
+    occ = []
+    for a, b in zip(edges[:-1], edges[1:]):
+        live = (start < b) & (end > a)
+        per_sm = np.bincount(rec["smid"][live], minlength=num_sms)
+        occ.append(round(float(per_sm.mean()), 2))
+    out["mean_ctas_per_sm_by_time_slice"] = occ
+    life = (end - start).sum()
+    out["share_of_cta_time_before_first_tile"] = float(np.nansum(first - start) / life)
+    ends = np.sort(end)
+    out["time_when_90pct_of_ctas_done_us"] = float(ends[int(0.9 * (len(ends) - 1))])
+    return out
+
+
+def main():
+    import json
+
+    import torch
+
+    import paged_kv_cache_475_b200 as pa
+    import workloads as W
+    from paged_kv_cache_475_b200.step import DecodeStep
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="llama_decode", choices=["llama_decode", "chat_trace", "long_context"])
+    ap.add_argument("--partition", default="auto")
+    ap.add_argument("--out", default=None)
+    a = ap.parse_args()
+    b = {"llama_decode": W.llama_decode, "chat_trace": W.chat_trace, "long_context": W.long_context}[a.workload](
+        poison=None).to("cuda")
+    sp = (b.info["shared_prefix_tokens"], b.info["shared_group"]) if a.workload == "chat_trace" else None
+    part = "auto" if a.partition == "auto" else (None if a.partition == "none" else int(a.partition))
+    step = DecodeStep(b.num_seqs, b.num_q_heads, b.num_kv_heads, b.head_dim, int(b.context_lens.max()), b.q.dtype,
+                      num_new_tokens=b.new_seq.shape[0], partition=part, shared_prefix=sp)
+    args = (b.q, b.k_new, b.v_new, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.new_seq, b.new_pos,
+            b.scale)
+    for _ in range(5):
+        step(*args)
+    torch.cuda.synchronize()
+    pa.trace_clear()
+    step(*args)
+    rec = pa.trace_read()
+    s = summarize(rec)
+    s["workload"] = a.workload
+    print(json.dumps(s))
+    if a.out:
+        np.savez(a.out, records=rec[rec["t_start"] > 0])
+
+
+if __name__ == "__main__":
+    main()
