@@ -45,17 +45,23 @@ namespace tc {
 constexpr int kM = 128;        // query rows per CTA = TMEM lanes
 constexpr int kN = 128;        // keys per tile
 #ifndef PA_TC_KSTAGES
-#define PA_TC_KSTAGES 2  // 3 measured slower (smaller L1 carve-out)
+#define PA_TC_KSTAGES 3  // a K slot takes ~2.4 us from free to landed (issue, then HBM); 3 stages hide it
 #endif
-#ifndef PA_TC_BT_PREFETCH
-#define PA_TC_BT_PREFETCH 0  // no measurable gain
+#ifndef PA_TC_BT_STAGED
+#define PA_TC_BT_STAGED 2048  // block-table entries staged in shared memory (32 768 tokens at B = 16)
 #endif
+constexpr int kBtStaged = PA_TC_BT_STAGED;
 constexpr int kStagesK = PA_TC_KSTAGES;  // K ring (S = Q K^T needs K earliest)
-constexpr int kStagesV = 2;    // V ring
-constexpr int kThreads = 352;  // 8 softmax warps + K producer + MMA + V producer
-constexpr int kProducerWarp = 8;   // Q once, then K tiles
+#ifndef PA_TC_VSTAGES
+#define PA_TC_VSTAGES 2
+#endif
+constexpr int kStagesV = PA_TC_VSTAGES;  // V ring
+constexpr int kThreads = 416;  // 8 softmax warps + MMA + 4 producers
+constexpr int kProducerWarp = 8;    // Q once, then the first half of every K tile's page chunks
 constexpr int kMmaWarp = 9;
-constexpr int kVProducerWarp = 10;  // V tiles
+constexpr int kVProducerWarp = 10;  // the first half of every V tile's page chunks
+constexpr int kKProducerWarp1 = 11; // the second half of the K chunks
+constexpr int kVProducerWarp1 = 12; // the second half of the V chunks
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;  // keep a stale max until the true one is 2^8 larger
@@ -79,6 +85,29 @@ struct Params {
   float* part_l;
   int part_np;
   int key_splits;
+  TraceRecord* trace;  // per-role timeline of one CTA (PA_TRACE builds), else null
+};
+
+// Per-role timeline events of the traced CTA (PA_TRACE builds): record index
+// event * 256 + tile, t_start = the global timer, kind = 100 + event.
+enum TraceEvent {
+  kEvKSlotFree = 0,  // K producer: slot free (empty barrier passed)
+  kEvKIssued,        // K producer: the tile's copies issued
+  kEvVSlotFree,      // V producer
+  kEvVIssued,
+  kEvMmaKFull,       // MMA: K tile landed
+  kEvMmaSIssued,     // MMA: S = Q K^T issued
+  kEvMmaVFull,       // MMA: V tile landed
+  kEvMmaP0,          // MMA: P of key half 0 ready
+  kEvMmaP1,          // MMA: P of key half 1 ready
+  kEvMmaPVIssued,    // MMA: both halves of P V issued
+  kEvSm0SFull,       // softmax warp 0 (rows 0..31, key half 0): S ready
+  kEvSm0PStored,     // softmax warp 0: P stored and signalled
+  kEvSm4SFull,       // softmax warp 4 (rows 0..31, key half 1)
+  kEvSm4PStored,
+  kEvKRowsDone,      // K producer: row coordinates of the tile computed
+  kEvKExpectDone,    // K producer: expect_tx armed, warp synchronised
+  kEvKAtom0Issued,   // K producer: copies of the first 64 columns issued
 };
 
 template <int D>
@@ -89,14 +118,18 @@ struct Smem {
   static constexpr int oK = oQ + kQ;
   static constexpr int oV = oK + kStagesK * kKV;
   static constexpr int oBar = oV + kStagesV * kKV;
-  // q_full, k_full/k_empty[SK], v_full/v_empty[SV], s_full[2], p_full[half][S buffer], o_done[half]
-  static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 2 + 4 + 2;
+  // q_full, k_full/k_empty[SK], v_full/v_empty[SV], s_full[2], p_full[half][S buffer], o_done[half], bt_ready
+  static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 2 + 4 + 2 + 1;
   static constexpr int oTmem = oBar + kNumBars * 8;
+  // The CTA's block-table entries, staged once: a producer's per-tile lookups
+  // then read shared memory instead of waiting on loads that queue behind the
+  // tiles' own traffic (about 1 us each under load).
+  static constexpr int oBt = (oTmem + 16 + 15) & ~15;
   // The epilogue's row-max / row-sum exchange reuses the Q tile, which no
   // MMA reads any more by then: [2 halves][128 rows] floats each.
   static constexpr int oRed = oQ;
   static constexpr int oSum = oQ + 1024;
-  static constexpr int kUsed = oTmem + 16;
+  static constexpr int kUsed = oBt + 4 * (kBtStaged > 0 ? kBtStaged : 1);
   static constexpr int kAlloc = kUsed + 1024;  // room to align the base to 1024 B
 };
 
@@ -346,10 +379,23 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // PV before writing P, can never be two phases ahead of the MMA's wait.
   uint64_t* p_full = s_full + 2;  // [2 halves][2 buffers]
   uint64_t* o_done = p_full + 4;  // [2]: PV of a key half done
+  uint64_t* bt_ready = o_done + 2;  // the staged block-table entries are in (32 arrivals)
+  int32_t* bt_s = reinterpret_cast<int32_t*>(smem + S::oBt);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::oTmem);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = gridDim.x - 1 - blockIdx.x;  // latest (heaviest) query tiles first
+#if PA_TRACE
+  // the traced CTA: the first dispatched (heaviest query tile) of sequence 0, KV head 0
+  const bool tr_on = p.trace != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+#define PA_TR(ev, j)                                                                                   \
+  do {                                                                                                 \
+    if (tr_on && lane == 0 && (j) < 256)                                                               \
+      p.trace[(ev) * 256 + (j)] = TraceRecord{global_ns(), 0, 0, sm_id(), (j), 0, 0, 0, 100 + (ev)};   \
+  } while (0)
+#else
+#define PA_TR(ev, j) do { } while (0)
+#endif
   const bool prefix_mode = p.prefix_len > 0;
   // prefix mode: z selects one of key_splits equal key ranges [key0, key0 + per)
   const int kvh = blockIdx.y, b = prefix_mode ? 0 : static_cast<int>(blockIdx.z);
@@ -373,11 +419,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < kStagesK; ++s) {
-      mbar_init(&k_full[s], 1);
+      mbar_init(&k_full[s], 2);  // the two K producer warps each arm their half
       mbar_init(&k_empty[s], 1);
     }
     for (int s = 0; s < kStagesV; ++s) {
-      mbar_init(&v_full[s], 1);
+      mbar_init(&v_full[s], 2);
       mbar_init(&v_empty[s], 1);
     }
     mbar_init(&s_full[0], 1);
@@ -387,6 +433,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       mbar_init(&p_full[2 * h + 1], 4);
       mbar_init(&o_done[h], 1);
     }
+    mbar_init(bt_ready, 32);
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -405,62 +452,86 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const uint32_t sQ = sb + S::oQ, sK = sb + S::oK, sV = sb + S::oV;
   const int32_t* bt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
 
-  if (warp == kProducerWarp || warp == kVProducerWarp) {
+  if (warp == kProducerWarp || warp == kVProducerWarp || warp == kKProducerWarp1 || warp == kVProducerWarp1) {
     // ------------------------- producers (K and V) -------------------------
-    // One warp per ring, so a K tile never waits for a V slot to free up.
-    const bool is_k = warp == kProducerWarp;
+    // Two warps per ring, each issuing the TMA boxes of half of a tile's page
+    // chunks, one box per lane: a warp issues its boxes one after another
+    // (about 45 ns each), so one warp per ring could not keep up with the
+    // tensor cores at 16-row pages (16 boxes per 128-key tile). Each warp arms
+    // its own half of the stage's bytes on the full barrier (2 arrivals).
+    const bool is_k = warp == kProducerWarp || warp == kKProducerWarp1;
+    const int half_id = (warp == kKProducerWarp1 || warp == kVProducerWarp1) ? 1 : 0;
     if (n_tiles > 0) {
-      if (is_k && lane == 0) {
+      if (warp == kProducerWarp && lane == 0) {
         mbar_arrive_expect_tx(q_full, S::kQ);
         for (int a = 0; a < KA; ++a)
           tma_load_3d(sQ + a * (kM * 128), &tm_q, a * 64, kvh * G, b * C + i0, q_full);
       }
       const int R = p.chunk_rows;
       const int chunks = kN / R;
+      const int half_chunks = chunks / 2;
       const int stages = is_k ? kStagesK : kStagesV;
+      int n_tiles_local = n_tiles;
       uint64_t* full = is_k ? k_full : v_full;
       uint64_t* empty = is_k ? k_empty : v_empty;
       const CUtensorMap* map = is_k ? &tm_k : &tm_v;
       const uint32_t ring = is_k ? sK : sV;
-      // Row coordinates of this lane's page chunks (c = lane, lane + 32) of
-      // tile j; the block-table reads for tile j + 1 are issued before the
-      // wait for tile j + 1's slot, so their latency hides behind it.
-      auto rows_of = [&](int j, int* y) {
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int c = lane + 32 * u;
-          const int t0 = key0 + j * kN + c * R;
-          y[u] = p.oob_row;  // chunks past the context read out of range: zeros
-          if (c < chunks && j < n_tiles && t0 < L) {
-            const int id = bt[t0 / B];
-            if (id >= 0 && id < p.num_blocks)
-              y[u] = (id * p.num_kv_heads + kvh) * B + (t0 % B);
-            else
-              set_error(p.err, PA_DEVERR_BLOCK_ID);
-          }
-        }
+      // The CTA's pages [jb0, jb0 + n_bt) as TMA row coordinates, staged
+      // once in shared memory (the first kBtStaged of them): row (id * Hkv +
+      // kvh) * B of the pool viewed as [P * Hkv * B, D], or -1 for a bad id.
+      // The first K producer's lanes fill it and each arrives on bt_ready
+      // after its own stores; the other producers wait for that.
+      const int jb0 = key0 / B;
+      const int k_end = min(L, key0 + n_tiles * kN);
+      const int n_bt = k_end > key0 ? (k_end - 1) / B - jb0 + 1 : 0;
+      const int n_staged = n_bt < kBtStaged ? n_bt : kBtStaged;
+      auto page_row = [&](int id) -> int {
+        if (id >= 0 && id < p.num_blocks) return (id * p.num_kv_heads + kvh) * B;
+        set_error(p.err, PA_DEVERR_BLOCK_ID);
+        return -1;
       };
-      int y_cur[2], y_next[2];
-      rows_of(0, y_cur);
-      for (int j = 0; j < n_tiles; ++j) {
+      if (warp == kProducerWarp) {
+        for (int i = lane; i < n_staged; i += 32) bt_s[i] = page_row(bt[jb0 + i]);
+        mbar_arrive(bt_ready);
+      } else if (!wait_all(bt_ready, 0)) {
+        if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
+        n_tiles_local = 0;
+      }
+      __syncwarp();
+      // This lane's box of every tile: page chunk c of this warp's half, atom a.
+      const bool has_box = lane < half_chunks * KA;
+      const int c = half_id * half_chunks + (has_box ? lane % half_chunks : 0);
+      const int a = has_box ? lane / half_chunks : 0;
+      const uint32_t half_bytes = static_cast<uint32_t>(half_chunks * R * D * 2);
+      // this lane's TMA row coordinate in tile j (the tile's page looked up
+      // in the staged entries, or in global memory past them)
+      auto row_of = [&](int j) -> int {
+        int y = p.oob_row;  // chunks past the context read out of range: zeros
+        const int t0 = key0 + j * kN + c * R;
+        if (has_box && j < n_tiles && t0 < L) {
+          const int jj = t0 / B - jb0;
+          const int row = jj < n_staged ? bt_s[jj] : page_row(bt[t0 / B]);
+          if (row >= 0) y = row + (t0 % B);
+        }
+        return y;
+      };
+      int y_next = row_of(0);
+      for (int j = 0; j < n_tiles_local; ++j) {
         const int st = j % stages;
-        if (PA_TC_BT_PREFETCH) rows_of(j + 1, y_next);
+        const int y = y_next;
+        y_next = row_of(j + 1);  // issued before the wait, so a global lookup's latency hides behind it
         if (!wait_all(&empty[st], ((j / stages) & 1) ^ 1)) {
           if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
           break;
         }
-        if (!PA_TC_BT_PREFETCH) rows_of(j, y_cur);
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], S::kKV);
+        if (half_id == 0) PA_TR(is_k ? kEvKSlotFree : kEvVSlotFree, j);
+        if (is_k && half_id == 0) PA_TR(kEvKRowsDone, j);
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], half_bytes);
         __syncwarp();
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int c = lane + 32 * u;
-          if (c < chunks)
-            for (int a = 0; a < KA; ++a)
-              tma_load_2d(ring + st * S::kKV + a * (kN * 128) + c * R * 128, map, a * 64, y_cur[u], &full[st]);
-        }
-        y_cur[0] = y_next[0];
-        y_cur[1] = y_next[1];
+        if (is_k && half_id == 0) PA_TR(kEvKExpectDone, j);
+        if (has_box) tma_load_2d(ring + st * S::kKV + a * (kN * 128) + c * R * 128, map, a * 64, y, &full[st]);
+        if (is_k && half_id == 0) PA_TR(kEvKAtom0Issued, j);
+        if (half_id == 0) PA_TR(is_k ? kEvKIssued : kEvVIssued, j);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -470,6 +541,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     auto issue_pv = [&](int k) -> bool {
       const int st = k % kStagesV;
       if (!wait_all(&v_full[st], (k / kStagesV) & 1)) return false;
+      PA_TR(kEvMmaVFull, k);
       // V rows past the context inside the last page chunk hold whatever the
       // pool holds there; P is 0 for them but 0 * NaN is NaN, so zero them.
       const int R = p.chunk_rows;
@@ -489,6 +561,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         if (!wait_all(&p_full[2 * h + (k & 1)], (k >> 1) & 1)) return false;
+        PA_TR(h ? kEvMmaP1 : kEvMmaP0, k);
         tc_fence_after();
         if (lane == 0) {
           // P of key half h sits in the first 32 columns of that half's S region
@@ -503,12 +576,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         __syncwarp();
       }
+      PA_TR(kEvMmaPVIssued, k);
       return true;
     };
     for (int j = 0; j < n_tiles && ok; ++j) {
       const int st = j % kStagesK;
       ok = wait_all(&k_full[st], (j / kStagesK) & 1);
       if (!ok) break;
+      PA_TR(kEvMmaKFull, j);
       tc_fence_after();
       if (lane == 0) {
         const uint32_t tS = (j & 1) ? tS1 : tS0;
@@ -524,6 +599,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc_commit(&k_empty[st]);
       }
       __syncwarp();
+      PA_TR(kEvMmaSIssued, j);
       if (j > 0) ok = issue_pv(j - 1);
     }
     if (ok && n_tiles > 0) ok = issue_pv(n_tiles - 1);
@@ -554,6 +630,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         ok = false;
         break;
       }
+      if (quad == 0) PA_TR(half ? kEvSm4SFull : kEvSm0SFull, j);
       tc_fence_after();
       float v[HC];
       {
@@ -636,6 +713,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[2 * half + (j & 1)]);
+      if (quad == 0) PA_TR(half ? kEvSm4PStored : kEvSm0PStored, j);
     }
     // epilogue: join the two halves, out = (O0 f0 + O1 f1) / (l0 f0 + l1 f1)
     bool got = ok;
@@ -810,6 +888,7 @@ int prefill_tcgen05(void* out, const void* q, const void* k_cache, const void* v
   prm.chunk_rows = block_size < 16 ? block_size : 16;
   prm.oob_row = static_cast<int>(pool_rows);  // first row past the pool: TMA reads zeros
   prm.scale_log2 = scale * tc::kLog2e;
+  prm.trace = trace_buffer();
   if (pp) {
     prm.prefix_len = pp->prefix_len;
     prm.part_o = pp->part_o;
