@@ -8,28 +8,29 @@
 // PagedAttention" (FlashAttention "Cómo funciona"); key tiles past a query
 // tile are never computed, the causal mask is applied in registers.
 //
-// One CTA (11 warps) per (sequence, KV head, 128-row query tile); the 128 rows
-// are (query, head) pairs of one GQA group, so each gathered K/V page serves
-// all G heads of the group. Warp roles:
-//   warps 0-7  softmax: warps w and w+4 own row block 32*(w%4).. (TMEM lanes);
-//              warp half h takes keys [64h, 64h+64) of every tile as its own
-//              online-softmax stream (own running max / sum, own TMEM O
-//              accumulator), writes its P (bf16/f16) back into TMEM over
-//              the S columns it read,
-//              rescales its O when its max grows by more than 2^8; the two
-//              streams are joined by the log-sum-exp rule when O is written;
-//   warps 8,10 producers: TMA tensor copies of the Q tile (once) and of each
-//              128-key K tile (warp 8) and V tile (warp 10, its own ring, so a K
-//              load never waits for a V slot), gathered page by page through
-//              the block table (one 2-D box of min(B,16) rows per page chunk,
-//              128-byte swizzle; chunks past the context read out of range
-//              and land as zeros);
-//   warp 9     MMA: one thread issues S = Q K^T into a double-buffered TMEM
-//              accumulator and O_h += P_h V_h per key half into two TMEM
-//              accumulators, P_h read straight from TMEM (A operand in tensor
-//              memory; M = 128, K = 16 per instruction), completions via tcgen05.commit
-//              on mbarriers; it zeroes V rows past the context in the last
-//              partial page chunk before they reach the PV product.
+// One CTA (7 warps) per (sequence, KV head, 128-row query tile), two CTAs per
+// SM; the 128 rows are (query, head) pairs of one GQA group, so each gathered
+// K/V page serves all G heads of the group. Warp roles:
+//   warps 0-3  softmax: warp w owns rows 32w.. (its TMEM lanes) and all 64 keys
+//              of every tile: one online-softmax stream per row (running max
+//              and sum in registers, O in TMEM), P (bf16/f16) written back into
+//              TMEM over the S columns it read, O rescaled only when the row
+//              max grows by more than 2^8;
+//   warps 4,6  producers: TMA tensor copies of the Q tile (once) and of each
+//              64-key K tile (warp 4) and V tile (warp 6, its own ring), one
+//              box per lane, addressed through the CTA's block-table entries
+//              staged once in shared memory as TMA row coordinates (one 2-D box
+//              of min(B,16) rows per page chunk and 128-byte atom, 128-byte
+//              swizzle; chunks past the context read out of range as zeros);
+//   warp 5     MMA: one thread issues S = Q K^T (M = 128, N = 64) into a
+//              double-buffered TMEM accumulator and O += P V (P read straight
+//              from TMEM as the A operand, K = 16 per instruction), completions
+//              by tcgen05.commit on mbarriers; it zeroes V rows past the context
+//              in the last partial page chunk before they reach the PV product.
+// A single CTA's tile chain is serial (S(j+2) needs PV(j), which needs the
+// softmax's P(j)), so each CTA holds half of what one CTA per SM would (256 TMEM
+// columns, 104 KB of shared memory) and the SM interleaves two such chains on
+// its tensor pipe.
 // Every mbarrier wait is bounded; a timeout sets PA_DEVERR_WAIT and the CTA
 // drains, frees its TMEM and returns.
 #include <cuda.h>
@@ -43,26 +44,19 @@ namespace pa {
 namespace tc {
 
 constexpr int kM = 128;        // query rows per CTA = TMEM lanes
-constexpr int kN = 128;        // keys per tile
-#ifndef PA_TC_KSTAGES
-#define PA_TC_KSTAGES 3  // a K slot takes ~2.4 us from free to landed (issue, then HBM); 3 stages hide it
-#endif
+constexpr int kN = 64;         // keys per tile
+constexpr int kStagesK = 2;    // K ring (16 KB per stage at D = 128)
+constexpr int kStagesV = 2;    // V ring
 #ifndef PA_TC_BT_STAGED
-#define PA_TC_BT_STAGED 2048  // block-table entries staged in shared memory (32 768 tokens at B = 16)
+#define PA_TC_BT_STAGED 1024  // block-table entries staged in shared memory (16 384 tokens at B = 16)
 #endif
 constexpr int kBtStaged = PA_TC_BT_STAGED;
-constexpr int kStagesK = PA_TC_KSTAGES;  // K ring (S = Q K^T needs K earliest)
-#ifndef PA_TC_VSTAGES
-#define PA_TC_VSTAGES 2
-#endif
-constexpr int kStagesV = PA_TC_VSTAGES;  // V ring
-constexpr int kThreads = 416;  // 8 softmax warps + MMA + 4 producers
-constexpr int kProducerWarp = 8;    // Q once, then the first half of every K tile's page chunks
-constexpr int kMmaWarp = 9;
-constexpr int kVProducerWarp = 10;  // the first half of every V tile's page chunks
-constexpr int kKProducerWarp1 = 11; // the second half of the K chunks
-constexpr int kVProducerWarp1 = 12; // the second half of the V chunks
-constexpr int kTmemCols = 512;
+constexpr int kThreads = 224;  // 4 softmax warps + K producer + MMA + V producer
+constexpr int kProducerWarp = 4;   // Q once, then K tiles
+constexpr int kMmaWarp = 5;
+constexpr int kVProducerWarp = 6;  // V tiles
+constexpr int kTmemCols = 256;     // S double buffer [0, 128), O [128, 128 + D); two CTAs share an SM's 512
+constexpr int kCtasPerSm = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;  // keep a stale max until the true one is 2^8 larger
 
@@ -98,12 +92,12 @@ enum TraceEvent {
   kEvMmaKFull,       // MMA: K tile landed
   kEvMmaSIssued,     // MMA: S = Q K^T issued
   kEvMmaVFull,       // MMA: V tile landed
-  kEvMmaP0,          // MMA: P of key half 0 ready
-  kEvMmaP1,          // MMA: P of key half 1 ready
+  kEvMmaP0,          // MMA: P ready
+  kEvMmaP1,          // (unused)
   kEvMmaPVIssued,    // MMA: both halves of P V issued
-  kEvSm0SFull,       // softmax warp 0 (rows 0..31, key half 0): S ready
+  kEvSm0SFull,       // softmax warp 0 (rows 0..31): S ready
   kEvSm0PStored,     // softmax warp 0: P stored and signalled
-  kEvSm4SFull,       // softmax warp 4 (rows 0..31, key half 1)
+  kEvSm4SFull,       // softmax warp 1 (rows 32..63)
   kEvSm4PStored,
   kEvKRowsDone,      // K producer: row coordinates of the tile computed
   kEvKExpectDone,    // K producer: expect_tx armed, warp synchronised
@@ -113,22 +107,16 @@ enum TraceEvent {
 template <int D>
 struct Smem {
   static constexpr int kQ = kM * D * 2;   // D/64 atoms of [128 rows x 128 B]
-  static constexpr int kKV = kN * D * 2;  // one K or V tile
+  static constexpr int kKV = kN * D * 2;  // one K or V tile: D/64 atoms of [64 rows x 128 B]
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + kQ;
   static constexpr int oV = oK + kStagesK * kKV;
   static constexpr int oBar = oV + kStagesV * kKV;
-  // q_full, k_full/k_empty[SK], v_full/v_empty[SV], s_full[2], p_full[half][S buffer], o_done[half], bt_ready
-  static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 2 + 4 + 2 + 1;
+  // q_full, k_full/k_empty[SK], v_full/v_empty[SV], s_full[2], p_full[2], o_done[2], bt_ready
+  static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 2 + 2 + 2 + 1;
   static constexpr int oTmem = oBar + kNumBars * 8;
-  // The CTA's block-table entries, staged once: a producer's per-tile lookups
-  // then read shared memory instead of waiting on loads that queue behind the
-  // tiles' own traffic (about 1 us each under load).
+  // The CTA's block-table entries as TMA row coordinates, staged once.
   static constexpr int oBt = (oTmem + 16 + 15) & ~15;
-  // The epilogue's row-max / row-sum exchange reuses the Q tile, which no
-  // MMA reads any more by then: [2 halves][128 rows] floats each.
-  static constexpr int oRed = oQ;
-  static constexpr int oSum = oQ + 1024;
   static constexpr int kUsed = oBt + 4 * (kBtStaged > 0 ? kBtStaged : 1);
   static constexpr int kAlloc = kUsed + 1024;  // room to align the base to 1024 B
 };
@@ -351,15 +339,15 @@ __device__ inline bool wait_all(uint64_t* bar, uint32_t parity) {
 }
 
 template <typename T, int D, int G>
-// 11 warps per CTA: the 4 SM sub-partitions hold 16K registers each and
-// three of them host 3 warps, so 168 registers per thread is the ceiling.
-__global__ void __launch_bounds__(kThreads, 1)
+// 7 warps per CTA, two CTAs per SM: 448 threads, so up to 146 registers each.
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const Params p) {
   using S = Smem<D>;
   constexpr int QT = kM / G;       // queries per CTA
   constexpr int KA = D / 64;       // 128-byte atoms along the head dim
   constexpr int KS = D / 16;       // MMA k-steps of S = Q K^T
+  constexpr int KP = kN / 16;      // MMA k-steps of O += P V
   constexpr uint32_t kIdescS = idesc_f16(Fmt<T>::kCode, 0, kM, kN);
   constexpr uint32_t kIdescO = idesc_f16(Fmt<T>::kCode, 1, kM, D);
 
@@ -373,12 +361,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   uint64_t* k_empty = k_full + kStagesK;
   uint64_t* v_full = k_empty + kStagesK;
   uint64_t* v_empty = v_full + kStagesV;
-  uint64_t* s_full = v_empty + kStagesV;  // [2]
-  // p_full[half][S buffer u]: P of tile 2n+u written (phase n), one barrier
-  // per buffer so that the softmax, which no longer waits for the previous
-  // PV before writing P, can never be two phases ahead of the MMA's wait.
-  uint64_t* p_full = s_full + 2;  // [2 halves][2 buffers]
-  uint64_t* o_done = p_full + 4;  // [2]: PV of a key half done
+  uint64_t* s_full = v_empty + kStagesV;  // [2]: S of tile 2n+u in buffer u (phase n)
+  // p_full[u]: P of tile 2n+u written over buffer u (phase n); one barrier per
+  // buffer, so the softmax can never be two phases ahead of the MMA's wait.
+  uint64_t* p_full = s_full + 2;
+  // o_done[u]: PV of tile 2n+u done (phase n). One barrier per buffer, like
+  // p_full: a waiter knows only that PV(j-2) is done when it waits for
+  // PV(j) (S(j) was issued after it), so with a single barrier it could be two
+  // phases behind and a parity wait would return on the older phase.
+  uint64_t* o_done = p_full + 2;
   uint64_t* bt_ready = o_done + 2;  // the staged block-table entries are in (32 arrivals)
   int32_t* bt_s = reinterpret_cast<int32_t*>(smem + S::oBt);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::oTmem);
@@ -419,20 +410,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < kStagesK; ++s) {
-      mbar_init(&k_full[s], 2);  // the two K producer warps each arm their half
+      mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
     }
     for (int s = 0; s < kStagesV; ++s) {
-      mbar_init(&v_full[s], 2);
+      mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
-    for (int h = 0; h < 2; ++h) {
-      mbar_init(&p_full[2 * h], 4);
-      mbar_init(&p_full[2 * h + 1], 4);
-      mbar_init(&o_done[h], 1);
-    }
+    mbar_init(&p_full[0], 4);
+    mbar_init(&p_full[1], 4);
+    mbar_init(&o_done[0], 1);
+    mbar_init(&o_done[1], 1);
     mbar_init(bt_ready, 32);
     fence_mbar_init();
   }
@@ -444,32 +434,27 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM columns: S (double buffer) [0, 256), O of key half 0 [256, 256 + D),
-  // O of key half 1 [256 + D, 256 + 2D).
+  // TMEM columns: S (double buffer) [0, 2 kN), O [2 kN, 2 kN + D).
   const uint32_t tS0 = tmem, tS1 = tmem + kN;
-  const uint32_t tO0 = tmem + 2 * kN, tO1 = tmem + 2 * kN + D;
+  const uint32_t tO = tmem + 2 * kN;
 
   const uint32_t sQ = sb + S::oQ, sK = sb + S::oK, sV = sb + S::oV;
   const int32_t* bt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
 
-  if (warp == kProducerWarp || warp == kVProducerWarp || warp == kKProducerWarp1 || warp == kVProducerWarp1) {
+  if (warp == kProducerWarp || warp == kVProducerWarp) {
     // ------------------------- producers (K and V) -------------------------
-    // Two warps per ring, each issuing the TMA boxes of half of a tile's page
-    // chunks, one box per lane: a warp issues its boxes one after another
-    // (about 45 ns each), so one warp per ring could not keep up with the
-    // tensor cores at 16-row pages (16 boxes per 128-key tile). Each warp arms
-    // its own half of the stage's bytes on the full barrier (2 arrivals).
-    const bool is_k = warp == kProducerWarp || warp == kKProducerWarp1;
-    const int half_id = (warp == kKProducerWarp1 || warp == kVProducerWarp1) ? 1 : 0;
+    // One warp per ring, one TMA box per lane: a tile is kN / R page chunks
+    // of R = min(B, 16) rows times D / 64 swizzle atoms, all issued by one
+    // warp instruction.
+    const bool is_k = warp == kProducerWarp;
     if (n_tiles > 0) {
-      if (warp == kProducerWarp && lane == 0) {
+      if (is_k && lane == 0) {
         mbar_arrive_expect_tx(q_full, S::kQ);
         for (int a = 0; a < KA; ++a)
           tma_load_3d(sQ + a * (kM * 128), &tm_q, a * 64, kvh * G, b * C + i0, q_full);
       }
       const int R = p.chunk_rows;
       const int chunks = kN / R;
-      const int half_chunks = chunks / 2;
       const int stages = is_k ? kStagesK : kStagesV;
       int n_tiles_local = n_tiles;
       uint64_t* full = is_k ? k_full : v_full;
@@ -479,8 +464,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       // The CTA's pages [jb0, jb0 + n_bt) as TMA row coordinates, staged
       // once in shared memory (the first kBtStaged of them): row (id * Hkv +
       // kvh) * B of the pool viewed as [P * Hkv * B, D], or -1 for a bad id.
-      // The first K producer's lanes fill it and each arrives on bt_ready
-      // after its own stores; the other producers wait for that.
+      // The K producer's lanes fill it and each arrives on bt_ready after its
+      // own stores; the V producer waits for that. Per-tile lookups then read
+      // shared memory instead of waiting on global loads that queue behind
+      // the tiles' own traffic.
       const int jb0 = key0 / B;
       const int k_end = min(L, key0 + n_tiles * kN);
       const int n_bt = k_end > key0 ? (k_end - 1) / B - jb0 + 1 : 0;
@@ -490,7 +477,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         set_error(p.err, PA_DEVERR_BLOCK_ID);
         return -1;
       };
-      if (warp == kProducerWarp) {
+      if (is_k) {
         for (int i = lane; i < n_staged; i += 32) bt_s[i] = page_row(bt[jb0 + i]);
         mbar_arrive(bt_ready);
       } else if (!wait_all(bt_ready, 0)) {
@@ -498,13 +485,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         n_tiles_local = 0;
       }
       __syncwarp();
-      // This lane's box of every tile: page chunk c of this warp's half, atom a.
-      const bool has_box = lane < half_chunks * KA;
-      const int c = half_id * half_chunks + (has_box ? lane % half_chunks : 0);
-      const int a = has_box ? lane / half_chunks : 0;
-      const uint32_t half_bytes = static_cast<uint32_t>(half_chunks * R * D * 2);
-      // this lane's TMA row coordinate in tile j (the tile's page looked up
-      // in the staged entries, or in global memory past them)
+      // This lane's box of every tile: page chunk c, atom a.
+      const bool has_box = lane < chunks * KA;
+      const int c = has_box ? lane % chunks : 0;
+      const int a = has_box ? lane / chunks : 0;
       auto row_of = [&](int j) -> int {
         int y = p.oob_row;  // chunks past the context read out of range: zeros
         const int t0 = key0 + j * kN + c * R;
@@ -524,20 +508,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
           break;
         }
-        if (half_id == 0) PA_TR(is_k ? kEvKSlotFree : kEvVSlotFree, j);
-        if (is_k && half_id == 0) PA_TR(kEvKRowsDone, j);
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], half_bytes);
+        PA_TR(is_k ? kEvKSlotFree : kEvVSlotFree, j);
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], S::kKV);
         __syncwarp();
-        if (is_k && half_id == 0) PA_TR(kEvKExpectDone, j);
         if (has_box) tma_load_2d(ring + st * S::kKV + a * (kN * 128) + c * R * 128, map, a * 64, y, &full[st]);
-        if (is_k && half_id == 0) PA_TR(kEvKAtom0Issued, j);
-        if (half_id == 0) PA_TR(is_k ? kEvKIssued : kEvVIssued, j);
+        PA_TR(is_k ? kEvKIssued : kEvVIssued, j);
       }
     }
   } else if (warp == kMmaWarp) {
     // -------------------------------- MMA ---------------------------------
     bool ok = n_tiles == 0 || wait_all(q_full, 0);
-    // PV of tile k, one key half at a time: O_h += P[:, half h] V[half h, :].
+    // PV of tile k: O += P V, P read from TMEM over the S columns of buffer k & 1.
     auto issue_pv = [&](int k) -> bool {
       const int st = k % kStagesV;
       if (!wait_all(&v_full[st], (k / kStagesV) & 1)) return false;
@@ -558,24 +539,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         fence_proxy_async_smem();
       }
       __syncwarp();
+      if (!wait_all(&p_full[k & 1], (k >> 1) & 1)) return false;
+      PA_TR(kEvMmaP0, k);
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t tP = (k & 1) ? tS1 : tS0;  // P (16-bit, two per column) over the first kN/2 columns
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (!wait_all(&p_full[2 * h + (k & 1)], (k >> 1) & 1)) return false;
-        PA_TR(h ? kEvMmaP1 : kEvMmaP0, k);
-        tc_fence_after();
-        if (lane == 0) {
-          // P of key half h sits in the first 32 columns of that half's S region
-          const uint32_t tP = ((k & 1) ? tS1 : tS0) + h * (kN / 2);
-#pragma unroll
-          for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
-            const uint64_t bd = sw128_desc(sV + st * S::kKV + kk * 2048, (kN * 128) >> 4, 64);
-            tc_mma_ts(h ? tO1 : tO0, tP + (kk % 4) * 8, bd, kIdescO, (k > 0 || kk > 4 * h) ? 1u : 0u);
-          }
-          tc_commit(&o_done[h]);
-          if (h == 1) tc_commit(&v_empty[st]);
+        for (int kk = 0; kk < KP; ++kk) {
+          const uint64_t bd = sw128_desc(sV + st * S::kKV + kk * 2048, (kN * 128) >> 4, 64);
+          tc_mma_ts(tO, tP + kk * 8, bd, kIdescO, (k > 0 || kk > 0) ? 1u : 0u);
         }
-        __syncwarp();
+        tc_commit(&o_done[k & 1]);
+        tc_commit(&v_empty[st]);
       }
+      __syncwarp();
       PA_TR(kEvMmaPVIssued, k);
       return true;
     };
@@ -606,23 +583,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (!ok && lane == 0) set_error(p.err, PA_DEVERR_WAIT);
   } else {
     // ------------------------------ softmax -------------------------------
-    // Warps w and w + 4 share TMEM lanes 32*(w%4).. (the rows). Warp half h
-    // takes keys [64h, 64h + 64) of every tile and runs its own online softmax
-    // over them (own running max / sum, own O accumulator, own P-ready and
-    // PV-done barriers), so the halves never wait for each other inside the
-    // loop; the epilogue joins the two streams with the log-sum-exp rule.
-    constexpr int HC = kN / 2;                 // key columns per half
-    constexpr int HD = D / 2;                  // output columns each half writes
-    const int quad = warp & 3, half = warp >> 2;
-    const int r = quad * 32 + lane;            // row = TMEM lane
+    // Warp w owns rows 32w..32w+31 (its TMEM lanes) and all kN keys of every
+    // tile: one online-softmax stream per row, running max and sum in
+    // registers, O in TMEM.
+    const int r = warp * 32 + lane;            // row = TMEM lane
     const int i = i0 + r / G, g = r % G;
     const int pos = prefix_mode ? L - 1 : L - C + i;
-    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const int bar_id = 1 + quad;
-    float* red = reinterpret_cast<float*>(smem + S::oRed);
-    float* rsum = reinterpret_cast<float*>(smem + S::oSum);
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-    const uint32_t tO = (half ? tO1 : tO0) + lane_off;
+    const uint32_t tOw = tO + lane_off;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
@@ -630,26 +599,26 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         ok = false;
         break;
       }
-      if (quad == 0) PA_TR(half ? kEvSm4SFull : kEvSm0SFull, j);
+      if (warp < 2) PA_TR(warp ? kEvSm4SFull : kEvSm0SFull, j);
       tc_fence_after();
-      float v[HC];
+      float v[kN];
       {
-        const uint32_t tS = ((j & 1) ? tS1 : tS0) + lane_off + half * HC;
-        tmem_ld32(tS, v);
-        tmem_ld32(tS + 32, v + 32);
+        const uint32_t tS = ((j & 1) ? tS1 : tS0) + lane_off;
+#pragma unroll
+        for (int cc = 0; cc < kN / 32; ++cc) tmem_ld32(tS + cc * 32, v + cc * 32);
         tmem_wait_ld();
       }
-      const int t0 = key0 + j * kN + half * HC;  // first key of this half
-      if (t0 + HC - 1 > pos_lo) {              // causal mask on the diagonal
+      const int t0 = key0 + j * kN;            // first key of the tile
+      if (t0 + kN - 1 > pos_lo) {              // causal mask on the diagonal
 #pragma unroll
-        for (int e = 0; e < HC; ++e)
+        for (int e = 0; e < kN; ++e)
           if (t0 + e > pos) v[e] = -INFINITY;
       }
       float mx8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx8[k] = v[k];
 #pragma unroll
-      for (int e = 8; e < HC; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], v[e]);
+      for (int e = 8; e < kN; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], v[e]);
 #pragma unroll
       for (int k = 0; k < 4; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + 4]);
       const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
@@ -662,12 +631,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float m_sub = m_use == -INFINITY ? 0.f : m_use;
       const float alpha = exp2f(m - m_sub);    // 0 while nothing was seen yet
       const float2 ms2 = make_float2(-m_sub, -m_sub);
-      uint32_t pk[HC / 2];
+      uint32_t pk[kN / 2];
       float2 ps2[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) ps2[k] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int e = 0; e < HC; e += 2) {
+      for (int e = 0; e < kN; e += 2) {
         const float2 x = __ffma2_rn(make_float2(v[e], v[e + 1]), sc2, ms2);
         const bool fma_path = ((e / 2) % 4) < PA_TC_POLY_OF_4;
         const uint32_t u = fma_path ? Fmt<T>::pack(ex2_sel<true>(x.x), ex2_sel<true>(x.y))
@@ -678,20 +647,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float2 pa2 = __fadd2_rn(__fadd2_rn(ps2[0], ps2[1]), __fadd2_rn(ps2[2], ps2[3]));
       l = l * alpha + (pa2.x + pa2.y);
       m = m_use;
-      // P goes back into TMEM over the first 32 columns of the S values this
+      // P goes back into TMEM over the first kN/2 columns of the S values this
       // warp just read (S buffer j&1; PV(j-2), the last reader of that buffer,
       // was issued before S(j), and tcgen05 MMAs run in issue order).
       {
-        const uint32_t tP = ((j & 1) ? tS1 : tS0) + lane_off + half * HC;
+        const uint32_t tP = ((j & 1) ? tS1 : tS0) + lane_off;
         tmem_st32(tP, reinterpret_cast<const float*>(pk));
       }
       if (j > 0) {
         // tcgen05.ld/st are warp-collective: the whole warp takes this branch
         // when any of its rows needs a rescale (the others multiply by 1). O
-        // may be touched only once PV(j-1) of this half is done.
+        // may be touched only once PV(j-1) is done.
         const bool need = rescale && alpha != 1.f;
         if (__any_sync(0xffffffffu, need)) {
-          if (!wait_all(&o_done[half], (j - 1) & 1)) {
+          if (!wait_all(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1)) {
             tmem_wait_st();
             ok = false;
             break;
@@ -699,79 +668,65 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           tc_fence_after();
           const float f = need ? alpha : 1.f;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int cc = 0; cc < D / 32; ++cc) {
             float o[32];
-            tmem_ld32(tO + c * 32, o);
+            tmem_ld32(tOw + cc * 32, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] *= f;
-            tmem_st32(tO + c * 32, o);
+            tmem_st32(tOw + cc * 32, o);
           }
         }
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[2 * half + (j & 1)]);
-      if (quad == 0) PA_TR(half ? kEvSm4PStored : kEvSm0PStored, j);
+      if (lane == 0) mbar_arrive(&p_full[j & 1]);
+      if (warp < 2) PA_TR(warp ? kEvSm4PStored : kEvSm0PStored, j);
     }
-    // epilogue: join the two halves, out = (O0 f0 + O1 f1) / (l0 f0 + l1 f1)
+    // epilogue: out = O / l (prefix mode: the unnormalised partial state)
     bool got = ok;
     if (ok && n_tiles > 0) {
-      got = wait_all(&o_done[half], (n_tiles - 1) & 1);
+      got = wait_all(&o_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);
       tc_fence_after();
     }
-    red[half * 128 + r] = m;
-    rsum[half * 128 + r] = l;
-    ok = pair_and(bar_id, 64, got);
-    if (!ok) {
+    if (!got) {
       if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
     } else {
-      const float m_o = red[(half ^ 1) * 128 + r], l_o = rsum[(half ^ 1) * 128 + r];
-      const float M = fmaxf(m, m_o);
-      const float Ms = M == -INFINITY ? 0.f : M;
-      const float f_self = exp2f(m - Ms), f_other = exp2f(m_o - Ms);
-      const float den = l * f_self + l_o * f_other;
-      const float f0 = half == 0 ? f_self : f_other, f1 = half == 0 ? f_other : f_self;
-      const float inv = (den > 0.f && n_tiles > 0) ? 1.f / den : 0.f;
-      // Every thread reads its O rows (warp-collective tcgen05.ld); only
-      // rows of real queries (i < C) are stored.
+      const float inv = (l > 0.f && n_tiles > 0) ? 1.f / l : 0.f;
+      // Every thread reads its O row (warp-collective tcgen05.ld); only rows
+      // of real queries (i < C) are stored.
       const bool store = i < C;
-      T* orow = static_cast<T*>(p.out) +
-                ((static_cast<int64_t>(b) * C + (store ? i : 0)) * p.num_q_heads + kvh * G + g) * D + half * HD;
-      // prefix mode: partial state of row (sequence i, head kvh*G + g), slot 0
+      T* orow = static_cast<T*>(p.out) + ((static_cast<int64_t>(b) * C + (store ? i : 0)) * p.num_q_heads + kvh * G + g) * D;
+      // prefix mode: partial state of row (sequence i, head kvh*G + g), slot `split`
       const int64_t prow = (static_cast<int64_t>(store ? i : 0) * p.num_q_heads + kvh * G + g) * p.part_np + split;
-      if (prefix_mode && store && half == 0) {
-        p.part_m[prow] = (den > 0.f && n_tiles > 0) ? Ms * 0.6931471805599453f : -INFINITY;
-        p.part_l[prow] = n_tiles > 0 ? den : 0.f;
+      if (prefix_mode && store) {
+        p.part_m[prow] = (l > 0.f && n_tiles > 0) ? m * 0.6931471805599453f : -INFINITY;
+        p.part_l[prow] = n_tiles > 0 ? l : 0.f;
       }
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        float o[32], o1[32];
+      for (int cc = 0; cc < D / 32; ++cc) {
+        float o[32];
         if (n_tiles > 0) {
-          tmem_ld32(tO0 + lane_off + half * HD + c * 32, o);
-          tmem_ld32(tO1 + lane_off + half * HD + c * 32, o1);
+          tmem_ld32(tOw + cc * 32, o);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = o1[e] = 0.f;
+          for (int e = 0; e < 32; ++e) o[e] = 0.f;
         }
         if (!store) continue;
-        if (prefix_mode) {  // unnormalised: sum_t 2^(s_t - M) v_t
-          float* dst = p.part_o + prow * D + half * HD + c * 32;
+        if (prefix_mode) {  // unnormalised: sum_t 2^(s_t - m) v_t
+          float* dst = p.part_o + prow * D + cc * 32;
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + e) = make_float4(o[e] * f0 + o1[e] * f1, o[e + 1] * f0 + o1[e + 1] * f1,
-                                                              o[e + 2] * f0 + o1[e + 2] * f1, o[e + 3] * f0 + o1[e + 3] * f1);
+            *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
           continue;
         }
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = (o[e] * f0 + o1[e] * f1) * inv;
-#pragma unroll
         for (int e = 0; e < 32; e += 8) {
-          uint4 w = make_uint4(Fmt<T>::pack_any(o[e], o[e + 1]), Fmt<T>::pack_any(o[e + 2], o[e + 3]),
-                               Fmt<T>::pack_any(o[e + 4], o[e + 5]), Fmt<T>::pack_any(o[e + 6], o[e + 7]));
-          *reinterpret_cast<uint4*>(orow + c * 32 + e) = w;
+          uint4 w = make_uint4(Fmt<T>::pack_any(o[e] * inv, o[e + 1] * inv), Fmt<T>::pack_any(o[e + 2] * inv, o[e + 3] * inv),
+                               Fmt<T>::pack_any(o[e + 4] * inv, o[e + 5] * inv), Fmt<T>::pack_any(o[e + 6] * inv, o[e + 7] * inv));
+          *reinterpret_cast<uint4*>(orow + cc * 32 + e) = w;
         }
       }
     }
@@ -835,9 +790,9 @@ int launch(const Params& prm, const void* q, const void* k_cache, const void* v_
     return record_cuda_error(cudaErrorInvalidValue, "prefill: encode v tensor map");
 
   auto kern = prefill_tc_kernel<T, D, G>;
-  // Above half of the SM's shared memory, so one CTA (and one TMEM allocation
-  // of 512 columns) per SM.
-  const int smem = Smem<D>::kAlloc > 120 * 1024 ? Smem<D>::kAlloc : 120 * 1024;
+  // At least a third of the SM's shared memory, so that at most two CTAs
+  // (two TMEM allocations of 256 columns) share an SM.
+  const int smem = Smem<D>::kAlloc > 78 * 1024 ? Smem<D>::kAlloc : 78 * 1024;
   // The attribute lives in the context: set it again after a device reset.
   static ContextCached<bool> attr_done[64];
   int dev = 0;
