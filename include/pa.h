@@ -342,6 +342,25 @@ PA_API int pa_decode_splitkv_noalloc(void* out, const void* q, const void* k_cac
                                      int partition_size, int num_partitions, float scale,
                                      pa_dtype dtype, void* stream);
 
+/*
+ * pa_decode_selftest_starved_wait - self-test of the copy-wait time-out; not
+ * part of the attention path. Runs pa_decode (same arguments, same checks)
+ * except that warp 0 of the first CTA arms its first copy stage for a tile
+ * whose copies are never issued, and every copy wait gives up after
+ * wait_cycles SM cycles (1000 .. 4e9; else PA_ERR_SHAPE). That wait runs out:
+ * the warp sets PA_DEVERR_WAIT, waits (same limit) for its copies that were
+ * issued, and the CTA finishes; rows of that CTA (KV head 0 of the longest
+ * sequence, the lowest index among equals; of sequence 0 when num_seqs is 1
+ * or above 512) are then undefined, all other rows are those of pa_decode. Nothing
+ * stays in flight, so the context remains usable. f16 with head_dim 128 only
+ * (else PA_ERR_UNSUPPORTED). Returns the launch status.
+ */
+PA_API int pa_decode_selftest_starved_wait(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                           const int32_t* block_tables, int max_blocks_per_seq,
+                                           const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                           int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                           float scale, pa_dtype dtype, long long wait_cycles, void* stream);
+
 /* Size in bytes of the per-device array pa_decode_splitkv_noalloc works in. */
 PA_API size_t pa_noalloc_scratch_bytes(void);
 
@@ -374,7 +393,8 @@ PA_API const char* pa_status_string(int status);
 PA_API int pa_trace_clear(void);
 PA_API int pa_trace_read(void* host_records, int max_records);
 
-/* Library ABI version (major * 100 + minor): 101 adds pa_splitkv_workspace_bytes. */
+/* Library ABI version (major * 100 + minor): 101 adds pa_splitkv_workspace_bytes,
+ * 102 pa_decode_selftest_starved_wait. */
 PA_API int pa_version(void);
 
 #ifdef __cplusplus

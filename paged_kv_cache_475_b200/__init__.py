@@ -40,6 +40,8 @@ _SIGS = {
     "pa_reshape_and_cache": [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp],
     "pa_copy_blocks": [_vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp],
     "pa_decode": [_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp],
+    "pa_decode_selftest_starved_wait": [_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _f, _i,
+                                        ctypes.c_longlong, _vp],
     "pa_decode_append": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp],
     "pa_decode_shared_prefix": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                                 _vp, _vp, _i, _f, _i, _vp],
@@ -209,6 +211,20 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float
     _check(_lib.pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                           block_tables.shape[1], _ptr(context_lens), N, q.shape[1], Hkv, D, B, P, float(scale),
                           _dtype_code(q), _stream(stream)), "pa_decode")
+
+
+def pa_decode_selftest_starved_wait(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                                    wait_cycles: int, stream=None):
+    """pa_decode with one copy wait that must time out (PA_DEVERR_WAIT); a self-test, not attention."""
+    _need(q, "q", None, 3)
+    _need(out, "out", q.dtype, 3)
+    P, Hkv, B, D, N = _cache_dims(q, k_cache, v_cache, block_tables, context_lens)
+    if q.shape[0] != N or q.shape[2] != D or out.shape != q.shape:
+        raise ValueError("q/out must be [N, Hq, D]")
+    _check(_lib.pa_decode_selftest_starved_wait(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), block_tables.shape[1],
+        _ptr(context_lens), N, q.shape[1], Hkv, D, B, P, float(scale), _dtype_code(q), int(wait_cycles),
+        _stream(stream)), "pa_decode_selftest_starved_wait")
 
 
 def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, scale: float,

@@ -133,7 +133,7 @@ extern "C" PA_API const char* pa_status_string(int status) {
   }
 }
 
-extern "C" PA_API int pa_version(void) { return 101; }
+extern "C" PA_API int pa_version(void) { return 102; }
 
 extern "C" PA_API int pa_splitkv_num_partitions(int max_context_len, int partition_size) {
   if (partition_size <= 0) return 0;

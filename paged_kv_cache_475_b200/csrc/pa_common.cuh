@@ -269,4 +269,13 @@ __device__ inline int sm_id() {
 // Packed fp32 FMA (sm_100): {a.x*b.x + c.x, a.y*b.y + c.y} in one instruction.
 __device__ inline float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
+// Maximum that returns NaN when either input is NaN (fmaxf returns the other
+// one), so that a NaN score or partial reaches the output as in the
+// definition of softmax attention instead of dropping out of a running max.
+__device__ inline float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
 }  // namespace pa

@@ -72,7 +72,7 @@ struct DecodeParams {
   int num_blocks;
   int partition;             // tokens per partition; 0 = whole sequence
   int num_parts;
-  int longest_first;         // map CTA z-index r to the r-th longest sequence
+  int longest_first;         // map CTA z-index r by longest-class-first order
   float q_scale;             // scale * log2(e)
   const void* k_new;         // fused append: [N, Hkv, D] rows of each sequence's newest token, or null
   const void* v_new;
@@ -84,44 +84,102 @@ struct DecodeParams {
   int cascade_group;
   int cascade_slot;
   TraceRecord* trace;        // timeline records (PA_TRACE builds), else null
+  // Read by the self-test instantiation only: copy-wait limit in SM cycles
+  // and, with starve_first_copy set, warp 0 of CTA (0, 0, 0) arms its first
+  // stage for a tile whose copies it never issues, so that wait must run out.
+  long long wait_cycles;
+  int starve_first_copy;
 };
 
-// Sequence whose work is the r-th largest (ties by index). CTAs are dispatched
-// in z order, so the longest contexts start first and short ones fill the
-// tail (greedy longest-processing-time scheduling). The CTA stages one 64-bit
-// key per sequence in shared memory (`keys`, room for the next power of two
-// >= n), high word the work + 2^31, low word the complement of the index, and
-// sorts them in descending order with a bitonic network: log2(n)(log2(n)+1)/2
-// compare-exchange rounds, n/2 pairs each, spread over the CTA's threads.
-// Work of sequence j is its length minus `skip` tokens when j < group.
-__device__ inline int longest_first_seq(const int32_t* lens, int n, int r, unsigned long long* keys, int group = 0,
-                                        int skip = 0) {
-  int n2 = 1;
-  while (n2 < n) n2 <<= 1;
-  for (int j = threadIdx.x; j < n2; j += blockDim.x) {
-    unsigned long long k = 0;  // padding sorts after every real key
-    if (j < n) {
-      const int w = lens[j] - (j < group ? skip : 0);
-      k = (static_cast<unsigned long long>(static_cast<unsigned>(w) + 0x80000000u) << 32) |
-          static_cast<unsigned long long>(0xffffffffu - static_cast<unsigned>(j));
-    }
-    keys[j] = k;
+#ifndef PA_DECODE_CLASS_BITS
+#define PA_DECODE_CLASS_BITS 2  // classes per octave of work: 2^bits
+#endif
+constexpr int kClassBits = PA_DECODE_CLASS_BITS;
+constexpr int kNumClasses = 32 << kClassBits;   // 128 (bits = 2) or 256 (bits = 3)
+constexpr int kClassesPerLane = kNumClasses / 32;
+
+// Work class of a sequence with work w: 2^bits * floor(log2 w) plus the
+// `bits` bits after the leading one (0 for w <= 0). Non-decreasing in w, so
+// classes split the lengths into 2^bits geometric bands per octave.
+__device__ inline int work_class(int w) {
+  if (w <= 0) return 0;
+  const unsigned u = static_cast<unsigned>(w);
+  const int e = 31 - __clz(u);
+  const unsigned mask = (1u << kClassBits) - 1u;
+  const unsigned m = e >= kClassBits ? (u >> (e - kClassBits)) & mask : (u << (kClassBits - e)) & mask;
+  return (e << kClassBits) + static_cast<int>(m);
+}
+
+// Sequence that CTA z-index r takes: classes in descending order, the
+// sequences of one class by index. CTAs are dispatched in z order, so the
+// longest contexts start first and short ones fill the tail (greedy
+// longest-processing-time scheduling, to within one class). Work of sequence
+// j is its length minus `skip` tokens when j < group. A counting sort: a
+// shared-memory histogram of the classes, one warp's scan of it to find the
+// class holding rank r and r's offset in it, then one warp's ballot walk
+// over the class bytes for that offset; three CTA barriers in all (an exact
+// bitonic sort of 256 keys takes 36, which on a batch of short sequences
+// cost a fifth of the step). `scratch` (the copy ring, not yet in use)
+// holds the counters, the answer and one class byte per sequence.
+__device__ inline int longest_class_first_seq(const int32_t* lens, int n, int r, int* scratch, int group = 0,
+                                              int skip = 0) {
+  int* cnt = scratch;                                                                // [kNumClasses]
+  int* answer = scratch + kNumClasses;                                               // [2]
+  unsigned char* cls = reinterpret_cast<unsigned char*>(scratch + kNumClasses + 2);  // [n]
+  for (int i = threadIdx.x; i < kNumClasses; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  for (int j = threadIdx.x; j < n; j += blockDim.x) {
+    const int c = work_class(lens[j] - (j < group ? skip : 0));
+    cls[j] = static_cast<unsigned char>(c);
+    atomicAdd(&cnt[c], 1);
   }
   __syncthreads();
-  for (int size = 2; size <= n2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int t = threadIdx.x; t < (n2 >> 1); t += blockDim.x) {
-        const int i = 2 * stride * (t / stride) + (t % stride);  // lower index of the pair
-        const unsigned long long a = keys[i], c = keys[i + stride];
-        if ((a < c) == ((i & size) == 0)) {  // descending blocks put the larger key first
-          keys[i] = c;
-          keys[i + stride] = a;
-        }
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    // lane l owns classes top - i, i = 0 .. kClassesPerLane - 1 (descending)
+    const int top = kNumClasses - 1 - kClassesPerLane * lane;
+    int c_own[kClassesPerLane], tot = 0;
+#pragma unroll
+    for (int i = 0; i < kClassesPerLane; ++i) {
+      c_own[i] = cnt[top - i];
+      tot += c_own[i];
+    }
+    int incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int start = incl - tot;  // sequences in the classes above this lane's
+    int my_cls = -1, my_off = 0;
+#pragma unroll
+    for (int i = 0; i < kClassesPerLane; ++i) {
+      if (r >= start && r < start + c_own[i]) {
+        my_cls = top - i;
+        my_off = r - start;
       }
-      __syncthreads();
+      start += c_own[i];
+    }
+    const unsigned who = __ballot_sync(0xffffffffu, my_cls >= 0);  // one lane, as 0 <= r < n
+    const int src = who ? __ffs(who) - 1 : 0;
+    const int want = __shfl_sync(0xffffffffu, my_cls, src);
+    int k = __shfl_sync(0xffffffffu, my_off, src);
+    if (lane == 0) answer[0] = r;  // kept only if r were out of range
+    __syncwarp();
+    for (int base = 0; base < n; base += 32) {
+      const int j = base + lane;
+      const bool in = j < n && cls[j] == want;
+      const unsigned m = __ballot_sync(0xffffffffu, in);
+      const int c = __popc(m);
+      if (k < c) {
+        if (in && __popc(m & ((1u << lane) - 1u)) == k) answer[0] = j;
+        break;
+      }
+      k -= c;
     }
   }
-  const int b = static_cast<int>(0xffffffffu - static_cast<unsigned>(keys[r] & 0xffffffffull));
+  __syncthreads();
+  const int b = answer[0];
   __syncthreads();  // the staging area is the copy ring, which the caller fills next
   return b;
 }
@@ -205,7 +263,7 @@ __device__ inline int head_src_lane(int g) {
   return lane;
 }
 
-struct MaxOp { __device__ float operator()(float a, float b) const { return fmaxf(a, b); } };
+struct MaxOp { __device__ float operator()(float a, float b) const { return fmax_nan(a, b); } };
 struct SumOp { __device__ float operator()(float a, float b) const { return a + b; } };
 
 template <typename T, int D, int G, int NW, int STAGES>
@@ -224,7 +282,7 @@ struct DecodeSmem {
 // No minimum-blocks bound: the fp16 / bf16 kernels at D = 128 fit three CTAs
 // per SM (167 registers, 67 KB) without one, and capping the registers at 170
 // to force it made the compiler trade ILP for registers (2.5% slower).
-template <typename T, int D, int G, int NW, int STAGES>
+template <typename T, int D, int G, int NW, int STAGES, bool kSelfTest = false>
 __global__ void __launch_bounds__(NW * 32, 1)
 decode_kernel(const DecodeParams p) {
   using S = DecodeShape<T, D, G>;
@@ -246,10 +304,9 @@ decode_kernel(const DecodeParams p) {
     if (threadIdx.x == 0 && kvh == 0 && p.context_lens[blockIdx.z] <= p.partition) set_error(p.err, PA_DEVERR_CONTEXT);
     return;
   }
-  const int b = p.longest_first
-                    ? longest_first_seq(p.context_lens, p.num_seqs, blockIdx.z,
-                                        reinterpret_cast<unsigned long long*>(smem), p.cascade_group,
-                                        p.cascade_prefix)
+const int b = p.longest_first
+                    ? longest_class_first_seq(p.context_lens, p.num_seqs, blockIdx.z, reinterpret_cast<int*>(smem),
+                                              p.cascade_group, p.cascade_prefix)
                     : static_cast<int>(blockIdx.z);
   const bool cascade_member = p.cascade_prefix > 0 && b < p.cascade_group;
   if (cascade_member && threadIdx.x == 0 && kvh == 0 && p.context_lens[b] <= p.cascade_prefix)
@@ -305,6 +362,12 @@ decode_kernel(const DecodeParams p) {
   load_ids(1, nxt0, nxt1);
   int ids_chunk = 0;
 
+  // Self-test instantiations only (a template flag, so that the attention
+  // kernels carry neither the check nor the limit in registers).
+  const bool starve = kSelfTest && p.starve_first_copy && warp == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&
+                      blockIdx.z == 0;
+  const long long wait_limit = kSelfTest ? p.wait_cycles : 4000000000LL;
+
   // Issue the copies of tile k into stage k % STAGES (all lanes call; lane 0 copies).
   auto issue = [&](int k) {
     const int chunk = k >> 5;
@@ -336,6 +399,8 @@ decode_kernel(const DecodeParams p) {
       if (!ok) {
         set_error(p.err, PA_DEVERR_BLOCK_ID);
         mbar_arrive_expect_tx(&bars[s], 0);
+      } else if (starve && k == 0) {
+        mbar_arrive_expect_tx(&bars[s], 2u * S::kTileBytes);  // no copy follows: the wait must time out
       } else if (B >= kTile) {
         const int64_t off = ((static_cast<int64_t>(id0) * p.num_kv_heads + kvh) * B + (t0 % B)) * D;
         mbar_arrive_expect_tx(&bars[s], 2u * S::kTileBytes);
@@ -426,7 +491,7 @@ decode_kernel(const DecodeParams p) {
   int k = 0;
   for (; k < my_tiles; ++k) {
     const int s = k % STAGES;
-    if (!__all_sync(0xffffffffu, mbar_wait(&bars[s], (k / STAGES) & 1))) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars[s], (k / STAGES) & 1, wait_limit))) {
       if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
       aborted = true;
       break;
@@ -478,14 +543,14 @@ decode_kernel(const DecodeParams p) {
         const int idx = base_idx + f;
         const int t = tg + S::kTG * (idx % S::kTPL);
         if (t >= nvalid) a[f] = -INFINITY;
-        vmax = fmaxf(vmax, a[f]);
+        vmax = fmax_nan(vmax, a[f]);
       }
       vmax = head_reduce<S::kNV, S::kDG, S::kTPL>(vmax, MaxOp());
       float alpha[G], m_use[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float tmax = __shfl_sync(0xffffffffu, vmax, head_src_lane<S::kNV, S::kDG, S::kTPL>(g));
-        const float m_new = fmaxf(m_run[g], tmax);
+        const float m_new = fmax_nan(m_run[g], tmax);
         m_use[g] = m_new == -INFINITY ? 0.f : m_new;
         alpha[g] = exp2f(m_run[g] - m_use[g]);  // exp2(-inf) = 0 on the first tile
         m_run[g] = m_new;
@@ -564,7 +629,8 @@ decode_kernel(const DecodeParams p) {
   if (aborted) {
     // Let this warp's copies still in flight land before the CTA exits.
     const int issued = my_tiles < k + STAGES ? my_tiles : k + STAGES;
-    for (int kk = k; kk < issued; ++kk) mbar_wait(&bars[kk % STAGES], (kk / STAGES) & 1, 400000000LL);
+    const long long drain_limit = kSelfTest ? p.wait_cycles : 400000000LL;
+    for (int kk = k; kk < issued; ++kk) mbar_wait(&bars[kk % STAGES], (kk / STAGES) & 1, drain_limit);
   }
 
   // ---- per-warp finish: l for every head -------------------------------------
@@ -593,7 +659,7 @@ decode_kernel(const DecodeParams p) {
     const int g = i / D, d = i % D;
     float Mx = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) Mx = fmaxf(Mx, mm[w * G + g]);
+    for (int w = 0; w < NW; ++w) Mx = fmax_nan(Mx, mm[w * G + g]);
     float o = 0.f, l = 0.f;
     if (Mx != -INFINITY) {
 #pragma unroll
@@ -616,7 +682,7 @@ decode_kernel(const DecodeParams p) {
       }
     } else {
       T* out = static_cast<T*>(p.out) + (static_cast<int64_t>(b) * p.num_q_heads + h) * D;
-      out[d] = Elem<T>::from_f(l > 0.f ? o / l : 0.f);
+      out[d] = Elem<T>::from_f(!(l <= 0.f) ? o / l : 0.f);  // l = NaN passes NaN on
     }
   }
 #if PA_TRACE
@@ -642,13 +708,13 @@ __device__ inline float block_reduce(float v, float* red, bool is_max) {
 #pragma unroll
   for (int off = 16; off >= 1; off /= 2) {
     const float o = __shfl_xor_sync(0xffffffffu, v, off);
-    v = is_max ? fmaxf(v, o) : v + o;
+    v = is_max ? fmax_nan(v, o) : v + o;
   }
   if (lane == 0) red[warp] = v;
   __syncthreads();
   float r = red[0];
 #pragma unroll
-  for (int w = 1; w < MW; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
+  for (int w = 1; w < MW; ++w) r = is_max ? fmax_nan(r, red[w]) : r + red[w];
   __syncthreads();
   return r;
 }
@@ -678,13 +744,13 @@ merge_kernel(T* __restrict__ out, const float* __restrict__ part_o, const float*
 
   float mloc = -INFINITY;
   for (int pp = threadIdx.x; pp < np; pp += MW * 32)
-    if (pl[pp] > 0.f) mloc = fmaxf(mloc, pm[pp]);
+    if (!(pl[pp] <= 0.f)) mloc = fmax_nan(mloc, pm[pp]);  // live: l > 0, or NaN (passed on)
   const float M = block_reduce<MW>(mloc, red, true);
   float dloc = 0.f;
   if (M != -INFINITY)
     for (int pp = threadIdx.x; pp < np; pp += MW * 32) {
       const float l = pl[pp];
-      dloc += l > 0.f ? expf(pm[pp] - M) * l : 0.f;
+      dloc += !(l <= 0.f) ? expf(pm[pp] - M) * l : 0.f;
     }
   const float den = block_reduce<MW>(dloc, red, false);
 
@@ -695,7 +761,7 @@ merge_kernel(T* __restrict__ out, const float* __restrict__ part_o, const float*
 #pragma unroll 4
     for (int pp = warp; pp < np; pp += MW) {
       const float l = pl[pp];
-      const float w = l > 0.f ? expf(pm[pp] - M) : 0.f;
+      const float w = !(l <= 0.f) ? expf(pm[pp] - M) : 0.f;
       float v[DPL];
       if constexpr (DPL == 4) {
         const float4 x = *reinterpret_cast<const float4*>(po + static_cast<int64_t>(pp) * D + lane * 4);
@@ -705,7 +771,7 @@ merge_kernel(T* __restrict__ out, const float* __restrict__ part_o, const float*
         v[0] = x.x; v[1] = x.y;
       }
 #pragma unroll
-      for (int j = 0; j < DPL; ++j) o[j] += l > 0.f ? w * v[j] : 0.f;
+      for (int j = 0; j < DPL; ++j) o[j] += !(l <= 0.f) ? w * v[j] : 0.f;
     }
   }
 #pragma unroll
@@ -715,7 +781,7 @@ merge_kernel(T* __restrict__ out, const float* __restrict__ part_o, const float*
     float num = 0.f;
 #pragma unroll
     for (int w = 0; w < MW; ++w) num += s_o[w][d];
-    out[static_cast<int64_t>(row) * D + d] = Elem<T>::from_f(den > 0.f ? num / den : 0.f);
+    out[static_cast<int64_t>(row) * D + d] = Elem<T>::from_f(!(den <= 0.f) ? num / den : 0.f);
   }
 }
 
@@ -730,17 +796,17 @@ merge_kernel(T* __restrict__ out, const float* __restrict__ part_o, const float*
 #define PA_DECODE_STAGES 2
 #endif
 #ifndef PA_DECODE_LPT_MAX_SEQS
-#define PA_DECODE_LPT_MAX_SEQS 512  // 512 x 8-byte keys fit the smallest copy ring (32 KB)
+#define PA_DECODE_LPT_MAX_SEQS 512  // class ordering stages n bytes + counters in the copy ring (>= 32 KB)
 #endif
 constexpr int kDecodeWarps = PA_DECODE_WARPS;
 constexpr int kDecodeStages = PA_DECODE_STAGES;
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, bool kSelfTest = false>
 int launch_decode(const DecodeParams& prm, int grid_x, cudaStream_t stream) {
   constexpr int NW = kDecodeWarps;
   constexpr int ST = (DecodeShape<T, D, G>::kTileBytes >= 8192 && kDecodeStages > 2) ? 2 : kDecodeStages;
   using M = DecodeSmem<T, D, G, NW, ST>;
-  auto kern = decode_kernel<T, D, G, NW, ST>;
+  auto kern = decode_kernel<T, D, G, NW, ST, kSelfTest>;
   // The attribute lives in the context: set it again after a device reset.
   static ContextCached<bool> attr_done[64];
   int dev = 0;
@@ -836,6 +902,49 @@ extern "C" PA_API int pa_decode(void* out, const void* q, const void* k_cache, c
   prm.num_parts = 1;
   prm.longest_first = num_seqs > 1 && num_seqs <= PA_DECODE_LPT_MAX_SEQS;
   return run_decode(prm, head_dim, scale, dtype, 1, (cudaStream_t)stream);
+}
+
+extern "C" PA_API int pa_decode_selftest_starved_wait(void* out, const void* q, const void* k_cache,
+                                                      const void* v_cache, const int32_t* block_tables,
+                                                      int max_blocks_per_seq, const int32_t* context_lens,
+                                                      int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                                      int block_size, int num_blocks, float scale, pa_dtype dtype,
+                                                      long long wait_cycles, void* stream) {
+  int st = check_decode_args(q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                             num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, dtype);
+  if (st != PA_OK || num_seqs == 0) return st;
+  if (!out) return PA_ERR_NULL;
+  if (num_seqs > 65535 || wait_cycles < 1000 || wait_cycles > 4000000000LL) return PA_ERR_SHAPE;
+  DecodeParams prm{};
+  prm.out = out;
+  prm.q = q;
+  prm.k_cache = k_cache;
+  prm.v_cache = v_cache;
+  prm.block_tables = block_tables;
+  prm.context_lens = context_lens;
+  prm.max_blocks = max_blocks_per_seq;
+  prm.num_seqs = num_seqs;
+  prm.num_q_heads = num_q_heads;
+  prm.num_kv_heads = num_kv_heads;
+  prm.block_size = block_size;
+  prm.num_blocks = num_blocks;
+  prm.partition = 0;
+  prm.num_parts = 1;
+  prm.longest_first = num_seqs > 1 && num_seqs <= PA_DECODE_LPT_MAX_SEQS;
+  prm.wait_cycles = wait_cycles;
+  prm.starve_first_copy = 1;
+  if (dtype != PA_F16 || head_dim != 128) return PA_ERR_UNSUPPORTED;  // the one instantiation kept for it
+  prm.q_scale = scale * kLog2e;
+  prm.err = device_error_word();
+  prm.trace = trace_buffer();
+  cudaStream_t s = (cudaStream_t)stream;
+  switch (num_q_heads / num_kv_heads) {
+    case 1: return launch_decode<__half, 128, 1, true>(prm, 1, s);
+    case 2: return launch_decode<__half, 128, 2, true>(prm, 1, s);
+    case 4: return launch_decode<__half, 128, 4, true>(prm, 1, s);
+    case 8: return launch_decode<__half, 128, 8, true>(prm, 1, s);
+  }
+  return PA_ERR_UNSUPPORTED;
 }
 
 extern "C" PA_API int pa_decode_append(void* out, const void* q, const void* k_new, const void* v_new,

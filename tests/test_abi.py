@@ -123,6 +123,17 @@ def test_decode_rejects_bad_args_on_host(lib, kw, code):
     assert lib.pa_decode(*_decode_args(**kw)) == code
 
 
+@pytest.mark.parametrize("cycles", [0, 999, 4_000_000_001, -5])
+def test_starved_wait_selftest_rejects_wait_limits_out_of_range_on_host(lib, cycles):
+    """The wait-limit self-test accepts 1000 .. 4e9 cycles and refuses the rest before any CUDA call."""
+    fn = lib.pa_decode_selftest_starved_wait
+    fn.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_void_p] + [ctypes.c_int] * 6 + [
+        ctypes.c_float, ctypes.c_int, ctypes.c_longlong, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    a = _decode_args()
+    assert fn(*a[:-1], cycles, None) == -2
+
+
 def test_splitkv_rejects_bad_partition(lib):
     fake = ctypes.c_void_p(16)
     args = [fake, fake, fake, fake, fake, fake, fake, 4, fake, 2, 8, 2, 128, 16, 10, 24, 3,

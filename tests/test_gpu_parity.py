@@ -413,3 +413,86 @@ def test_decode_shared_prefix_rejects_a_member_inside_the_prefix():
     b = small_batch(seed=410, lens=(64, 100, 300), shared_prefix_tokens=64, shared_group=2)
     out, _, flags = run_gpu(b, shared_prefix="batch")   # sequence 0 ends exactly at the prefix end
     assert flags & pa.DEVERR_CONTEXT
+
+
+# ---------------------------------------------------------------------------
+# Copy-wait time-out
+# ---------------------------------------------------------------------------
+
+def test_copy_wait_times_out_sets_the_flag_and_the_context_stays_usable():
+    """A wait for a copy that is never issued gives up, reports PA_DEVERR_WAIT and leaves nothing in flight.
+
+    The self-test entry point arms warp 0 of the first CTA (KV head 0 of the longest sequence) for a tile
+    whose copies never come, with a wait limit of 2e5 SM cycles (about 0.1 ms). Every other CTA runs as in
+    pa_decode, so every other row must equal pa_decode's bit for bit; a plain decode afterwards must match
+    the oracle with no flag set.
+    """
+    import paged_kv_cache_475_b200 as pa
+    b = small_batch(seed=420, lens=(1, 15, 100, 700, 333, 17), poison=None)  # unique longest: sequence 3
+    g = b.to("cuda")
+    pa.pa_read_error_flags(clear=True)
+    ref_gpu = torch.empty_like(g.q)
+    pa.pa_decode(ref_gpu, g.q, g.k_cache, g.v_cache, g.block_tables, g.context_lens, g.scale)
+    assert pa.pa_read_error_flags() == 0
+
+    starved = torch.full_like(g.q, float("nan"))
+    pa.pa_decode_selftest_starved_wait(starved, g.q, g.k_cache, g.v_cache, g.block_tables, g.context_lens,
+                                       g.scale, wait_cycles=200_000)
+    assert pa.pa_read_error_flags(clear=True) == pa.DEVERR_WAIT
+    G = g.q.shape[1] // g.k_cache.shape[1]
+    keep = torch.ones(g.q.shape[:2], dtype=torch.bool, device="cuda")
+    keep[3, :G] = False
+    assert torch.equal(starved[keep].view(torch.int16), ref_gpu[keep].view(torch.int16))
+
+    again = torch.empty_like(g.q)
+    pa.pa_decode(again, g.q, g.k_cache, g.v_cache, g.block_tables, g.context_lens, g.scale)
+    assert pa.pa_read_error_flags() == 0
+    assert torch.equal(again.view(torch.int16), ref_gpu.view(torch.int16))
+    expect = oracle.attention(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.scale)
+    assert_close(again, expect, "f16", "decode after a timed-out wait")
+
+
+# ---------------------------------------------------------------------------
+# Non-finite values inside the visible context
+# ---------------------------------------------------------------------------
+
+def _plant(cache, bt, seq, pos, kvh, d, B):
+    cache[int(bt[seq, pos // B]), kvh, pos % B, d] = float("nan")
+
+
+def test_nan_in_a_visible_key_or_value_reaches_the_output_as_in_the_definition():
+    """A NaN in a visible K row makes every score of that KV head's rows NaN, so the whole rows are NaN; a
+    NaN in a visible V element makes that output dimension NaN. The oracle (the plain definition) says so;
+    the kernels must agree, also where the NaN key is the only token of a warp's tiles (position 16 of a
+    17-token context, position 0 of a 1-token one), through the single pass and through split-KV + merge.
+    """
+    import paged_kv_cache_475_b200 as pa
+    b = small_batch(seed=421, lens=(1, 17, 40, 300, 64), poison=None)
+    B = b.block_size
+    _plant(b.k_cache, b.block_tables, 0, 0, 0, 5, B)      # sequence 0, its only key, KV head 0
+    _plant(b.k_cache, b.block_tables, 1, 16, 1, 77, B)    # sequence 1, key 16 (alone in its tile), KV head 1
+    _plant(b.v_cache, b.block_tables, 3, 123, 0, 9, B)    # sequence 3, value 123, KV head 0, dim 9
+    expect = oracle.attention(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.scale)
+    assert np.isnan(expect[0, :4]).all() and np.isnan(expect[1, 4:]).all()
+    assert np.isnan(expect[3, :4, 9]).all() and np.isfinite(np.delete(expect[3, :4], 9, axis=-1)).all()
+    g = b.to("cuda")
+    pa.pa_read_error_flags(clear=True)
+    single = torch.empty_like(g.q)
+    pa.pa_decode(single, g.q, g.k_cache, g.v_cache, g.block_tables, g.context_lens, g.scale)
+    outs = {"single pass": single}
+    for partition in (16, 128):
+        nparts = pa.pa_splitkv_num_partitions(int(b.context_lens.max()), partition)
+        po, pm, pl = pa.splitkv_buffers(b.num_seqs, b.num_q_heads, b.head_dim, nparts)
+        merged = torch.empty_like(g.q)
+        pa.pa_decode_splitkv(po, pm, pl, g.q, g.k_cache, g.v_cache, g.block_tables, g.context_lens, partition,
+                             g.scale)
+        pa.pa_merge(merged, po, pm, pl, g.context_lens, partition)
+        outs[f"split {partition}"] = merged
+    torch.cuda.synchronize()
+    assert pa.pa_read_error_flags() == 0
+    nan = np.isnan(expect)
+    for what, out in outs.items():
+        got = out.cpu().to(torch.float64).numpy()
+        assert (np.isnan(got) == nan).all(), f"{what}: NaN pattern differs from the definition"
+        err = np.abs(got[~nan] - expect[~nan])
+        assert err.max() <= 1e-2 and err.mean() <= 1e-3, f"{what}: finite part off by {err.max():.3e}"
