@@ -253,6 +253,11 @@ constexpr int kTraceMax = 1 << 16;
 // Device address of the record array (lives in pa_api.cu; every .cu is its own
 // device module, so kernels get the address as a parameter); null unless PA_TRACE.
 TraceRecord* trace_buffer();
+
+// Merge of split-KV partials (pa_merge.cu) on `s`, for `rows` = N * Hq rows;
+// partition < 0: the first -partition slots of each row are live.
+int launch_merge_any(void* out, const float* po, const float* pm, const float* pl, const int32_t* lens, int rows,
+                     int Hq, int D, int partition, int np, pa_dtype dt, cudaStream_t s);
 #if PA_TRACE
 __device__ inline unsigned long long global_ns() {
   unsigned long long t;
