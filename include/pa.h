@@ -84,6 +84,8 @@ typedef enum {
 #define PA_DEVERR_SLOT 0x4u        /* slot_mapping entry outside the pool */
 #define PA_DEVERR_WAIT 0x8u        /* an asynchronous copy did not land within its wait limit */
 #define PA_DEVERR_POSITION 0x10u   /* slot mapping: sequence index or position outside the table */
+#define PA_DEVERR_SETUP 0x20u      /* a CTA could not set itself up (its shared-memory base not at the
+                                      alignment its tensor copies need) and computed nothing */
 
 /*
  * pa_slot_mapping - flat cache slot of each new token.

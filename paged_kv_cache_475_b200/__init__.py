@@ -32,6 +32,7 @@ DEVERR_CONTEXT = 0x2
 DEVERR_SLOT = 0x4
 DEVERR_WAIT = 0x8
 DEVERR_POSITION = 0x10
+DEVERR_SETUP = 0x20
 
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 

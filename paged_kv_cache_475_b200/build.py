@@ -59,11 +59,15 @@ def _stale(defines=()) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, defines=(), lib: str = LIB, objdir: str = BUILD) -> str:
+def build(force: bool = False, verbose: bool = False, defines=None, lib: str = LIB, objdir: str = BUILD) -> str:
     """Compile every CUDA source for sm_100a and link libpa.so; returns its path.
 
-    defines: extra -D macros (tuning variants), written to `lib` with objects in `objdir`.
+    defines: extra -D macros (tuning variants), written to `lib` with objects in `objdir`; None takes
+    them from the PA_BUILD_DEFINES environment variable (space-separated, empty by default), so that
+    a variant built that way is not rebuilt by a later plain build() in the same environment.
     """
+    if defines is None:
+        defines = tuple(os.environ.get("PA_BUILD_DEFINES", "").split())
     if not force and os.path.abspath(lib) == LIB and not _stale(tuple(defines)):
         return LIB
     os.makedirs(objdir, exist_ok=True)

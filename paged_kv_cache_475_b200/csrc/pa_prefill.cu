@@ -19,9 +19,10 @@
 //   warps 4,6  producers: TMA tensor copies of the Q tile (once) and of each
 //              64-key K tile (warp 4) and V tile (warp 6, its own ring), one
 //              box per lane, addressed through the CTA's block-table entries
-//              staged once in shared memory as TMA row coordinates (one 2-D box
+//              (the first 128 staged once in shared memory as TMA row
+//              coordinates, later ones read one tile ahead) with one 2-D box
 //              of min(B,16) rows per page chunk and 128-byte atom, 128-byte
-//              swizzle; chunks past the context read out of range as zeros);
+//              swizzle; chunks past the context read out of range as zeros;
 //   warp 5     MMA: one thread issues S = Q K^T (M = 128, N = 64) into a
 //              double-buffered TMEM accumulator and O += P V (P read straight
 //              from TMEM as the A operand, K = 16 per instruction), completions
@@ -29,8 +30,11 @@
 //              in the last partial page chunk before they reach the PV product.
 // A single CTA's tile chain is serial (S(j+2) needs PV(j), which needs the
 // softmax's P(j)), so each CTA holds half of what one CTA per SM would (256 TMEM
-// columns, 104 KB of shared memory) and the SM interleaves two such chains on
-// its tensor pipe.
+// columns, 97 KB of shared memory) and the SM interleaves two such chains on
+// its tensor pipe. Per 64-key tile the MMA thread issues 12 instructions of
+// 24-47 ns of tensor work each, and issuing them takes about 0.7 us of the
+// ~1.25 us tile period: with tiles this size the issuing thread, not the
+// tensor pipe, sets the pace.
 // Every mbarrier wait is bounded; a timeout sets PA_DEVERR_WAIT and the CTA
 // drains, frees its TMEM and returns.
 #include <cuda.h>
@@ -45,10 +49,20 @@ namespace tc {
 
 constexpr int kM = 128;        // query rows per CTA = TMEM lanes
 constexpr int kN = 64;         // keys per tile
-constexpr int kStagesK = 2;    // K ring (16 KB per stage at D = 128)
-constexpr int kStagesV = 2;    // V ring
+#ifndef PA_TC_KSTAGES
+#define PA_TC_KSTAGES 2
+#endif
+#ifndef PA_TC_VSTAGES
+#define PA_TC_VSTAGES 2
+#endif
+#ifndef PA_TC_SMEM_SLACK
+#define PA_TC_SMEM_SLACK 0  // bytes reserved to align the dynamic shared-memory base at run time (the base
+                            // measured 1024-aligned; the kernel checks it and reports PA_DEVERR_SETUP if not)
+#endif
+constexpr int kStagesK = PA_TC_KSTAGES;  // K ring (16 KB per stage at D = 128)
+constexpr int kStagesV = PA_TC_VSTAGES;  // V ring
 #ifndef PA_TC_BT_STAGED
-#define PA_TC_BT_STAGED 1024  // block-table entries staged in shared memory (16 384 tokens at B = 16)
+#define PA_TC_BT_STAGED 128  // block-table entries staged in shared memory (2048 tokens at B = 16; 1024 measured 1.6% slower)
 #endif
 constexpr int kBtStaged = PA_TC_BT_STAGED;
 constexpr int kThreads = 224;  // 4 softmax warps + K producer + MMA + V producer
@@ -118,7 +132,7 @@ struct Smem {
   // The CTA's block-table entries as TMA row coordinates, staged once.
   static constexpr int oBt = (oTmem + 16 + 15) & ~15;
   static constexpr int kUsed = oBt + 4 * (kBtStaged > 0 ? kBtStaged : 1);
-  static constexpr int kAlloc = kUsed + 1024;  // room to align the base to 1024 B
+  static constexpr int kAlloc = kUsed + PA_TC_SMEM_SLACK;  // room to align the base to 1024 B
 };
 
 // ---------------------------------------------------------------------------
@@ -351,8 +365,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   constexpr uint32_t kIdescS = idesc_f16(Fmt<T>::kCode, 0, kM, kN);
   constexpr uint32_t kIdescO = idesc_f16(Fmt<T>::kCode, 1, kM, D);
 
-  extern __shared__ unsigned char smem_raw[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
+  // The 128-byte-swizzled tiles need a 1024-byte-aligned base. Without the
+  // slack to align it here, a base that is not aligned is reported and the
+  // CTA does nothing (checked before any shared memory or TMEM is touched).
+  if (PA_TC_SMEM_SLACK < 1024 && (raw_addr & 1023u) != 0u) {
+    if (threadIdx.x == 0) set_error(p.err, PA_DEVERR_SETUP);
+    return;
+  }
   unsigned char* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const uint32_t sb = smem_addr(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::oBar);
