@@ -74,6 +74,9 @@ struct DecodeParams {
   int partition;             // tokens per partition; 0 = whole sequence
   int num_parts;
   int longest_first;         // map CTA z-index r by longest-class-first order
+  // Row pairing (single pass only; 0: off): CTAs with z >= pair_from take two
+  // rows, ranks pair_from + 2 (z - pair_from) and the next one, two warps each.
+  int pair_from;
   float q_scale;             // scale * log2(e)
   const void* k_new;         // fused append: [N, Hkv, D] rows of each sequence's newest token, or null
   const void* v_new;
@@ -111,8 +114,9 @@ __device__ inline int work_class(int w) {
   return (e << kClassBits) + static_cast<int>(m);
 }
 
-// Sequence that CTA z-index r takes: classes in descending order, the
-// sequences of one class by index. CTAs are dispatched in z order, so the
+// Sequences of ranks r0 and r1 (r1 < 0: none) in this order: classes in
+// descending order, the sequences of one class by index; -1 for a rank
+// outside [0, n). CTAs are dispatched in z order, so the
 // longest contexts start first and short ones fill the tail (greedy
 // longest-processing-time scheduling, to within one class). Work of sequence
 // j is its length minus `skip` tokens when j < group. A counting sort: a
@@ -122,8 +126,8 @@ __device__ inline int work_class(int w) {
 // bitonic sort of 256 keys takes 36, which on a batch of short sequences
 // cost a fifth of the step). `scratch` (the copy ring, not yet in use)
 // holds the counters, the answer and one class byte per sequence.
-__device__ inline int longest_class_first_seq(const int32_t* lens, int n, int r, int* scratch, int group = 0,
-                                              int skip = 0) {
+__device__ inline void longest_class_first_seqs(const int32_t* lens, int n, int r0, int r1, int* scratch, int group,
+                                                int skip, int* b0, int* b1) {
   int* cnt = scratch;                                                                // [kNumClasses]
   int* answer = scratch + kNumClasses;                                               // [2]
   unsigned char* cls = reinterpret_cast<unsigned char*>(scratch + kNumClasses + 2);  // [n]
@@ -151,38 +155,43 @@ __device__ inline int longest_class_first_seq(const int32_t* lens, int n, int r,
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += v;
     }
-    int start = incl - tot;  // sequences in the classes above this lane's
-    int my_cls = -1, my_off = 0;
+    const int start0 = incl - tot;  // sequences in the classes above this lane's
+    for (int t = 0; t < 2; ++t) {
+      const int r = t ? r1 : r0;
+      if (lane == 0) answer[t] = -1;  // no rank (r < 0 or r >= n): an empty row slot
+      __syncwarp();
+      if (r < 0 || r >= n) continue;
+      int my_cls = -1, my_off = 0;
+      int st = start0;
 #pragma unroll
-    for (int i = 0; i < kClassesPerLane; ++i) {
-      if (r >= start && r < start + c_own[i]) {
-        my_cls = top - i;
-        my_off = r - start;
+      for (int i = 0; i < kClassesPerLane; ++i) {
+        if (r >= st && r < st + c_own[i]) {
+          my_cls = top - i;
+          my_off = r - st;
+        }
+        st += c_own[i];
       }
-      start += c_own[i];
-    }
-    const unsigned who = __ballot_sync(0xffffffffu, my_cls >= 0);  // one lane, as 0 <= r < n
-    const int src = who ? __ffs(who) - 1 : 0;
-    const int want = __shfl_sync(0xffffffffu, my_cls, src);
-    int k = __shfl_sync(0xffffffffu, my_off, src);
-    if (lane == 0) answer[0] = r;  // kept only if r were out of range
-    __syncwarp();
-    for (int base = 0; base < n; base += 32) {
-      const int j = base + lane;
-      const bool in = j < n && cls[j] == want;
-      const unsigned m = __ballot_sync(0xffffffffu, in);
-      const int c = __popc(m);
-      if (k < c) {
-        if (in && __popc(m & ((1u << lane) - 1u)) == k) answer[0] = j;
-        break;
+      const unsigned who = __ballot_sync(0xffffffffu, my_cls >= 0);  // one lane, as 0 <= r < n
+      const int src = who ? __ffs(who) - 1 : 0;
+      const int want = __shfl_sync(0xffffffffu, my_cls, src);
+      int k = __shfl_sync(0xffffffffu, my_off, src);
+      for (int base = 0; base < n; base += 32) {
+        const int j = base + lane;
+        const bool in = j < n && cls[j] == want;
+        const unsigned m = __ballot_sync(0xffffffffu, in);
+        const int c = __popc(m);
+        if (k < c) {
+          if (in && __popc(m & ((1u << lane) - 1u)) == k) answer[t] = j;
+          break;
+        }
+        k -= c;
       }
-      k -= c;
     }
   }
   __syncthreads();
-  const int b = answer[0];
+  *b0 = answer[0];
+  *b1 = answer[1];
   __syncthreads();  // the staging area is the copy ring, which the caller fills next
-  return b;
 }
 
 // Reduce-scatter of a[NV] over the kDG lanes of a token group (xor offsets
@@ -305,18 +314,34 @@ decode_kernel(const DecodeParams p) {
     if (threadIdx.x == 0 && kvh == 0 && p.context_lens[blockIdx.z] <= p.partition) set_error(p.err, PA_DEVERR_CONTEXT);
     return;
   }
-const int b = p.longest_first
-                    ? longest_class_first_seq(p.context_lens, p.num_seqs, blockIdx.z, reinterpret_cast<int*>(smem),
-                                              p.cascade_group, p.cascade_prefix)
-                    : static_cast<int>(blockIdx.z);
-  const bool cascade_member = p.cascade_prefix > 0 && b < p.cascade_group;
-  if (cascade_member && threadIdx.x == 0 && kvh == 0 && p.context_lens[b] <= p.cascade_prefix)
+  // Rows of this CTA: one, or two short ones (ranks past the longest
+  // pair_from) with NW/2 warps each. Warp `warp` works on row `sub` as warp
+  // `wr` of the row's `wpr`; a row slot past the batch (b < 0) is empty.
+  const int z = static_cast<int>(blockIdx.z);
+  const bool paired = !split && p.pair_from > 0 && z >= p.pair_from;
+  const int wpr = paired ? NW / 2 : NW;
+  const int sub = warp / wpr;
+  const int wr = warp - sub * wpr;
+  const int r0 = paired ? p.pair_from + 2 * (z - p.pair_from) : z;
+  const int r1 = paired ? r0 + 1 : -1;
+  int b_row0, b_row1;
+  if (p.longest_first) {
+    longest_class_first_seqs(p.context_lens, p.num_seqs, r0, r1, reinterpret_cast<int*>(smem), p.cascade_group,
+                             p.cascade_prefix, &b_row0, &b_row1);
+  } else {
+    b_row0 = r0 < p.num_seqs ? r0 : -1;
+    b_row1 = (r1 >= 0 && r1 < p.num_seqs) ? r1 : -1;
+  }
+  const int b = sub ? b_row1 : b_row0;
+  const bool row_lead = wr == 0 && lane == 0;  // reports this row's errors
+  const bool cascade_member = p.cascade_prefix > 0 && b >= 0 && b < p.cascade_group;
+  if (cascade_member && row_lead && kvh == 0 && p.context_lens[b] <= p.cascade_prefix)
     set_error(p.err, PA_DEVERR_CONTEXT);
 
-  // ---- context range of this CTA -------------------------------------------
-  int L = p.context_lens[b];
+  // ---- context range of this warp's row --------------------------------------
+  int L = b >= 0 ? p.context_lens[b] : 0;
   if (L < 0 || L > p.max_blocks * p.block_size) {
-    if (threadIdx.x == 0) set_error(p.err, PA_DEVERR_CONTEXT);
+    if (row_lead) set_error(p.err, PA_DEVERR_CONTEXT);
     L = L < 0 ? 0 : p.max_blocks * p.block_size;
   }
   if (split && part == p.num_parts - 1 && L > p.num_parts * p.partition && threadIdx.x == 0)
@@ -325,7 +350,7 @@ const int b = p.longest_first
   int t_end = split ? min(L, t_begin + p.partition) : L;
   if (t_end < t_begin) t_end = t_begin;
   const int n_tiles = (t_end - t_begin + kTile - 1) / kTile;
-  const int my_tiles = warp < n_tiles ? (n_tiles - warp + NW - 1) / NW : 0;
+  const int my_tiles = wr < n_tiles ? (n_tiles - wr + wpr - 1) / wpr : 0;
 
   unsigned char* ring = smem + warp * STAGES * M::kStageBytes;
   float* prob = reinterpret_cast<float*>(smem + M::kDataBytes) + warp * kTile * G;
@@ -340,7 +365,7 @@ const int b = p.longest_first
 
   const T* kc = static_cast<const T*>(p.k_cache);
   const T* vc = static_cast<const T*>(p.v_cache);
-  const int32_t* bt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
+  const int32_t* bt = p.block_tables + static_cast<int64_t>(b < 0 ? 0 : b) * p.max_blocks;
   const int B = p.block_size;
   const int n_seq_blocks = (L + B - 1) / B;
 
@@ -352,7 +377,7 @@ const int b = p.longest_first
     id0 = -1;
     id1 = -1;
     if (k < my_tiles) {
-      const int t0 = t_begin + (warp + NW * k) * kTile;
+      const int t0 = t_begin + (wr + wpr * k) * kTile;
       const int j = t0 / B;
       id0 = bt[j];
       if (B < kTile && j + 1 < n_seq_blocks && t0 + B < t_end) id1 = bt[j + 1];
@@ -382,7 +407,7 @@ const int b = p.longest_first
     const int id1 = __shfl_sync(0xffffffffu, cur1, k & 31);
     if (lane == 0) {
       const int s = k % STAGES;
-      const int t0 = t_begin + (warp + NW * k) * kTile;
+      const int t0 = t_begin + (wr + wpr * k) * kTile;
       const int nvalid = min(kTile, t_end - t0);
       unsigned char* kdst = ring + s * M::kStageBytes;
       unsigned char* vdst = kdst + S::kTileBytes;
@@ -427,7 +452,7 @@ const int b = p.longest_first
   const int tg = lane / S::kDG;
   float2 q2[G][S::kQPL / 2];
   {
-    const T* qb = static_cast<const T*>(p.q) + (static_cast<int64_t>(b) * p.num_q_heads + kvh * G) * D;
+    const T* qb = static_cast<const T*>(p.q) + (static_cast<int64_t>(b < 0 ? 0 : b) * p.num_q_heads + kvh * G) * D;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
 #pragma unroll
@@ -464,7 +489,7 @@ const int b = p.longest_first
   // fence by every writing lane and a warp barrier, so that lane 0's bulk
   // copies (async proxy) see the row.
   if (p.k_new != nullptr && L > 0 && t_begin <= L - 1 && L - 1 < t_end &&
-      warp == ((L - 1 - t_begin) / kTile) % NW) {
+      wr == ((L - 1 - t_begin) / kTile) % wpr) {
     const int pos = L - 1;
     const int phys = bt[pos / B];
     if (phys >= 0 && phys < p.num_blocks) {
@@ -656,15 +681,18 @@ const int b = p.longest_first
   }
   __syncthreads();
 
-  for (int i = threadIdx.x; i < G * D; i += NW * 32) {
-    const int g = i / D, d = i % D;
+  const int n_rows = paired ? 2 : 1;
+  for (int i = threadIdx.x; i < n_rows * G * D; i += NW * 32) {
+    const int rs = i / (G * D);  // row slot: its warps are rs * wpr .. rs * wpr + wpr - 1
+    const int g = (i / D) % G, d = i % D;
+    const int rb = rs ? b_row1 : b_row0;
+    if (rb < 0) continue;
+    const int w0 = rs * wpr;
     float Mx = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) Mx = fmax_nan(Mx, mm[w * G + g]);
+    for (int w = w0; w < w0 + wpr; ++w) Mx = fmax_nan(Mx, mm[w * G + g]);
     float o = 0.f, l = 0.f;
     if (Mx != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < NW; ++w) {
+      for (int w = w0; w < w0 + wpr; ++w) {
         const float mw = mm[w * G + g];
         if (mw == -INFINITY) continue;
         const float sc = exp2f(mw - Mx);
@@ -673,16 +701,17 @@ const int b = p.longest_first
       }
     }
     const int h = kvh * G + g;
-    if (split || cascade_member) {
+    const bool member = p.cascade_prefix > 0 && rb < p.cascade_group;
+    if (split || member) {
       const int slot = split ? part : p.cascade_slot;
-      const int64_t row = (static_cast<int64_t>(b) * p.num_q_heads + h) * p.num_parts + slot;
+      const int64_t row = (static_cast<int64_t>(rb) * p.num_q_heads + h) * p.num_parts + slot;
       p.part_o[row * D + d] = o;
       if (d == 0) {
         p.part_m[row] = Mx == -INFINITY ? -INFINITY : Mx * kLn2;
         p.part_l[row] = l;
       }
     } else {
-      T* out = static_cast<T*>(p.out) + (static_cast<int64_t>(b) * p.num_q_heads + h) * D;
+      T* out = static_cast<T*>(p.out) + (static_cast<int64_t>(rb) * p.num_q_heads + h) * D;
       out[d] = Elem<T>::from_f(!(l <= 0.f) ? o / l : 0.f);  // l = NaN passes NaN on
     }
   }
@@ -730,7 +759,8 @@ int launch_decode(const DecodeParams& prm, int grid_x, cudaStream_t stream) {
     if (e != cudaSuccess) return record_cuda_error(e, "decode: set the shared memory carveout");
     if (dev >= 0 && dev < 64) attr_done[dev].set(true);
   }
-  dim3 grid(grid_x, prm.num_kv_heads, prm.num_seqs);
+  const int grid_z = prm.pair_from > 0 ? prm.pair_from + (prm.num_seqs - prm.pair_from + 1) / 2 : prm.num_seqs;
+  dim3 grid(grid_x, prm.num_kv_heads, grid_z);
   kern<<<grid, NW * 32, M::kTotal, stream>>>(prm);
   return launch_status();
 }
@@ -751,6 +781,36 @@ int dispatch_dim(const DecodeParams& prm, int D, int G, int grid_x, cudaStream_t
   if (D == 64) return dispatch_group<T, 64>(prm, G, grid_x, s);
   if (D == 128) return dispatch_group<T, 128>(prm, G, grid_x, s);
   return PA_ERR_UNSUPPORTED;
+}
+
+#ifndef PA_DECODE_PAIR_WAVES
+#define PA_DECODE_PAIR_WAVES 3  // pair rows when one row per CTA would take more waves than this (0: never)
+#endif
+#ifndef PA_DECODE_PAIR_KEEP_DIV
+#define PA_DECODE_PAIR_KEEP_DIV 8  // the longest num_seqs / this ranks keep a CTA each (4 and 2 measured slower)
+#endif
+
+// Rank from which a single-pass launch gives each CTA two rows (0: none).
+// Only a batch whose one-row-per-CTA grid would take more than
+// PA_DECODE_PAIR_WAVES waves of three CTAs per SM is paired: there the CTAs
+// are short and their start-up (ordering, block ids, first copies) is a
+// large share of their life, so two rows with two warps each per CTA keep
+// twice as many rows in flight per SM. The longest num_seqs / KEEP_DIV
+// ranks (the first CTAs in longest-class-first order) keep all four warps.
+int decode_pair_from(int num_seqs, int num_kv_heads) {
+  if (PA_DECODE_PAIR_WAVES <= 0 || num_seqs < 2) return 0;
+  static int sms[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int n_sm = dev >= 0 && dev < 64 ? sms[dev] : 0;
+  if (n_sm <= 0) {
+    if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) return 0;
+    if (dev >= 0 && dev < 64) sms[dev] = n_sm;
+  }
+  const long long ctas = static_cast<long long>(num_seqs) * num_kv_heads;
+  if (ctas <= static_cast<long long>(PA_DECODE_PAIR_WAVES) * 3 * n_sm) return 0;
+  const int keep = num_seqs / PA_DECODE_PAIR_KEEP_DIV;
+  return keep < 1 ? 1 : keep;
 }
 
 int run_decode(DecodeParams prm, int D, float scale, pa_dtype dt, int grid_x, cudaStream_t s) {
@@ -812,6 +872,7 @@ extern "C" PA_API int pa_decode(void* out, const void* q, const void* k_cache, c
   prm.partition = 0;
   prm.num_parts = 1;
   prm.longest_first = num_seqs > 1 && num_seqs <= PA_DECODE_LPT_MAX_SEQS;
+  prm.pair_from = decode_pair_from(num_seqs, num_kv_heads);
   return run_decode(prm, head_dim, scale, dtype, 1, (cudaStream_t)stream);
 }
 
@@ -842,6 +903,7 @@ extern "C" PA_API int pa_decode_selftest_starved_wait(void* out, const void* q, 
   prm.partition = 0;
   prm.num_parts = 1;
   prm.longest_first = num_seqs > 1 && num_seqs <= PA_DECODE_LPT_MAX_SEQS;
+  prm.pair_from = decode_pair_from(num_seqs, num_kv_heads);
   prm.wait_cycles = wait_cycles;
   prm.starve_first_copy = 1;
   if (dtype != PA_F16 || head_dim != 128) return PA_ERR_UNSUPPORTED;  // the one instantiation kept for it
@@ -1072,6 +1134,7 @@ extern "C" PA_API int pa_decode_shared_prefix(void* out, const void* q, const vo
   prm.cascade_group = group_size;
   prm.cascade_slot = splits;
   prm.longest_first = num_seqs > 1 && num_seqs <= PA_DECODE_LPT_MAX_SEQS;
+  prm.pair_from = decode_pair_from(num_seqs, num_kv_heads);
   st = run_decode(prm, head_dim, scale, dtype, 1, s);
   if (group_size == 0) return st;
   const cudaError_t e = cudaStreamWaitEvent(s, side->join, 0);  // join, whatever happened above

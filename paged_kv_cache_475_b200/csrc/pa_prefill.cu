@@ -19,10 +19,11 @@
 //   warps 4,6  producers: TMA tensor copies of the Q tile (once) and of each
 //              64-key K tile (warp 4) and V tile (warp 6, its own ring), one
 //              box per lane, addressed through the CTA's block-table entries
-//              (the first 128 staged once in shared memory as TMA row
-//              coordinates, later ones read one tile ahead) with one 2-D box
-//              of min(B,16) rows per page chunk and 128-byte atom, 128-byte
-//              swizzle; chunks past the context read out of range as zeros;
+//              (each read one tile ahead of its copy; PA_TC_BT_STAGED > 0
+//              stages the first ones in shared memory instead, measured
+//              slower) with one 2-D box of min(B,16) rows per page chunk and
+//              128-byte atom, 128-byte swizzle; chunks past the context read
+//              out of range as zeros;
 //   warp 5     MMA: one thread issues S = Q K^T (M = 128, N = 64) into a
 //              double-buffered TMEM accumulator and O += P V (P read straight
 //              from TMEM as the A operand, K = 16 per instruction), completions
@@ -30,7 +31,7 @@
 //              in the last partial page chunk before they reach the PV product.
 // A single CTA's tile chain is serial (S(j+2) needs PV(j), which needs the
 // softmax's P(j)), so each CTA holds half of what one CTA per SM would (256 TMEM
-// columns, 97 KB of shared memory) and the SM interleaves two such chains on
+// columns, 96 KB of shared memory) and the SM interleaves two such chains on
 // its tensor pipe. Per 64-key tile the MMA thread issues 12 instructions of
 // 24-47 ns of tensor work each, and issuing them takes about 0.7 us of the
 // ~1.25 us tile period: with tiles this size the issuing thread, not the
@@ -62,7 +63,7 @@ constexpr int kN = 64;         // keys per tile
 constexpr int kStagesK = PA_TC_KSTAGES;  // K ring (16 KB per stage at D = 128)
 constexpr int kStagesV = PA_TC_VSTAGES;  // V ring
 #ifndef PA_TC_BT_STAGED
-#define PA_TC_BT_STAGED 128  // block-table entries staged in shared memory (2048 tokens at B = 16; 1024 measured 1.6% slower)
+#define PA_TC_BT_STAGED 0  // block-table entries staged in shared memory (0: each read one tile ahead; 128 / 256 / 1024 measured 1 / 2 / 3% slower)
 #endif
 constexpr int kBtStaged = PA_TC_BT_STAGED;
 constexpr int kThreads = 224;  // 4 softmax warps + K producer + MMA + V producer

@@ -496,3 +496,40 @@ def test_nan_in_a_visible_key_or_value_reaches_the_output_as_in_the_definition()
         assert (np.isnan(got) == nan).all(), f"{what}: NaN pattern differs from the definition"
         err = np.abs(got[~nan] - expect[~nan])
         assert err.max() <= 1e-2 and err.mean() <= 1e-3, f"{what}: finite part off by {err.max():.3e}"
+
+
+# ---------------------------------------------------------------------------
+# Two rows per CTA (large batches of mostly short rows)
+# ---------------------------------------------------------------------------
+
+def _paired_lens(seed, n):
+    g = np.random.default_rng(seed)
+    lens = g.integers(1, 400, n)
+    lens[:5] = (1, 2, 15, 16, 17)
+    return tuple(int(x) for x in lens)
+
+
+@pytest.mark.parametrize("fused", [True, False])
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_decode_with_paired_rows(dtype, fused):
+    """300 sequences x 8 KV heads is more than three waves of CTAs on a B200, so the single pass gives the
+    CTAs past the longest eighth two rows each (two warps per row); 300 - 37 = 263 paired ranks leave the
+    last CTA one empty row slot. Every row must match the oracle and the cache write must be bit-exact."""
+    b = small_batch(seed=430, dtype=dtype, G=4, Hkv=8, B=16, lens=_paired_lens(430, 300))
+    ref, kc, vc, _ = oracle.step(b)
+    out, g, flags = run_gpu(b, partition=None, fused_append=fused)
+    assert flags == 0
+    assert_close(out, ref, dtype, f"paired rows {dtype} fused={fused}")
+    assert torch.equal(g.k_cache.cpu().view(torch.int16), kc.view(torch.int16))
+    assert torch.equal(g.v_cache.cpu().view(torch.int16), vc.view(torch.int16))
+
+
+def test_shared_prefix_with_paired_rows():
+    """The cascade's suffix pass pairs rows too: members (suffix only) and non-members mixed in pairs."""
+    lens = tuple(64 + x if i < 120 else x for i, x in enumerate(_paired_lens(431, 300)))
+    b = small_batch(seed=431, dtype="f16", G=4, Hkv=8, B=16, lens=lens, shared_prefix_tokens=64, shared_group=120)
+    ref, kc, vc, _ = oracle.step(b)
+    out, g, flags = run_gpu(b, fused_append=True, shared_prefix="batch")
+    assert flags == 0
+    assert_close(out, ref, "f16", "shared prefix with paired rows")
+    assert torch.equal(g.k_cache.cpu().view(torch.int16), kc.view(torch.int16))
