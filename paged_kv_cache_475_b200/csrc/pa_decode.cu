@@ -26,6 +26,7 @@
 //    lane owning D/32 output dims for all G heads;
 //  * the warps' (m, l, o) states merge in shared memory at the end.
 #include <mutex>
+#include <type_traits>
 
 #include "pa_common.cuh"
 
@@ -126,6 +127,7 @@ __device__ inline int work_class(int w) {
 // bitonic sort of 256 keys takes 36, which on a batch of short sequences
 // cost a fifth of the step). `scratch` (the copy ring, not yet in use)
 // holds the counters, the answer and one class byte per sequence.
+template <bool kTwo>
 __device__ inline void longest_class_first_seqs(const int32_t* lens, int n, int r0, int r1, int* scratch, int group,
                                                 int skip, int* b0, int* b1) {
   int* cnt = scratch;                                                                // [kNumClasses]
@@ -156,7 +158,7 @@ __device__ inline void longest_class_first_seqs(const int32_t* lens, int n, int 
       if (lane >= o) incl += v;
     }
     const int start0 = incl - tot;  // sequences in the classes above this lane's
-    for (int t = 0; t < 2; ++t) {
+    for (int t = 0; t < (kTwo ? 2 : 1); ++t) {
       const int r = t ? r1 : r0;
       if (lane == 0) answer[t] = -1;  // no rank (r < 0 or r >= n): an empty row slot
       __syncwarp();
@@ -190,7 +192,7 @@ __device__ inline void longest_class_first_seqs(const int32_t* lens, int n, int 
   }
   __syncthreads();
   *b0 = answer[0];
-  *b1 = answer[1];
+  *b1 = kTwo ? answer[1] : -1;
   __syncthreads();  // the staging area is the copy ring, which the caller fills next
 }
 
@@ -292,7 +294,7 @@ struct DecodeSmem {
 // No minimum-blocks bound: the fp16 / bf16 kernels at D = 128 fit three CTAs
 // per SM (167 registers, 67 KB) without one, and capping the registers at 170
 // to force it made the compiler trade ILP for registers (2.5% slower).
-template <typename T, int D, int G, int NW, int STAGES, bool kSelfTest = false>
+template <typename T, int D, int G, int NW, int STAGES, bool kSelfTest = false, bool kPaired = false>
 __global__ void __launch_bounds__(NW * 32, 1)
 decode_kernel(const DecodeParams p) {
   using S = DecodeShape<T, D, G>;
@@ -318,7 +320,10 @@ decode_kernel(const DecodeParams p) {
   // pair_from) with NW/2 warps each. Warp `warp` works on row `sub` as warp
   // `wr` of the row's `wpr`; a row slot past the batch (b < 0) is empty.
   const int z = static_cast<int>(blockIdx.z);
-  const bool paired = !split && p.pair_from > 0 && z >= p.pair_from;
+  // Pairing is a separate instantiation (kPaired), so that every other
+  // launch keeps the fixed one-row layout (its divisions by constants, its
+  // unrolled merge); a paired launch's first pair_from CTAs take one row.
+  const bool paired = kPaired && !split && p.pair_from > 0 && z >= p.pair_from;
   const int wpr = paired ? NW / 2 : NW;
   const int sub = warp / wpr;
   const int wr = warp - sub * wpr;
@@ -326,8 +331,8 @@ decode_kernel(const DecodeParams p) {
   const int r1 = paired ? r0 + 1 : -1;
   int b_row0, b_row1;
   if (p.longest_first) {
-    longest_class_first_seqs(p.context_lens, p.num_seqs, r0, r1, reinterpret_cast<int*>(smem), p.cascade_group,
-                             p.cascade_prefix, &b_row0, &b_row1);
+    longest_class_first_seqs<kPaired>(p.context_lens, p.num_seqs, r0, r1, reinterpret_cast<int*>(smem),
+                                      p.cascade_group, p.cascade_prefix, &b_row0, &b_row1);
   } else {
     b_row0 = r0 < p.num_seqs ? r0 : -1;
     b_row1 = (r1 >= 0 && r1 < p.num_seqs) ? r1 : -1;
@@ -689,10 +694,15 @@ decode_kernel(const DecodeParams p) {
     if (rb < 0) continue;
     const int w0 = rs * wpr;
     float Mx = -INFINITY;
-    for (int w = w0; w < w0 + wpr; ++w) Mx = fmax_nan(Mx, mm[w * G + g]);
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+      if (!kPaired || w < wpr) Mx = fmax_nan(Mx, mm[(w0 + w) * G + g]);
     float o = 0.f, l = 0.f;
     if (Mx != -INFINITY) {
-      for (int w = w0; w < w0 + wpr; ++w) {
+#pragma unroll
+      for (int ww = 0; ww < NW; ++ww) {
+        if (kPaired && ww >= wpr) break;
+        const int w = w0 + ww;
         const float mw = mm[w * G + g];
         if (mw == -INFINITY) continue;
         const float sc = exp2f(mw - Mx);
@@ -741,12 +751,12 @@ decode_kernel(const DecodeParams p) {
 constexpr int kDecodeWarps = PA_DECODE_WARPS;
 constexpr int kDecodeStages = PA_DECODE_STAGES;
 
-template <typename T, int D, int G, bool kSelfTest = false>
+template <typename T, int D, int G, bool kSelfTest = false, bool kPaired = false>
 int launch_decode(const DecodeParams& prm, int grid_x, cudaStream_t stream) {
   constexpr int NW = kDecodeWarps;
   constexpr int ST = (DecodeShape<T, D, G>::kTileBytes >= 8192 && kDecodeStages > 2) ? 2 : kDecodeStages;
   using M = DecodeSmem<T, D, G, NW, ST>;
-  auto kern = decode_kernel<T, D, G, NW, ST, kSelfTest>;
+  auto kern = decode_kernel<T, D, G, NW, ST, kSelfTest, kPaired>;
   // The attribute lives in the context: set it again after a device reset.
   static ContextCached<bool> attr_done[64];
   int dev = 0;
@@ -767,11 +777,25 @@ int launch_decode(const DecodeParams& prm, int grid_x, cudaStream_t stream) {
 
 template <typename T, int D>
 int dispatch_group(const DecodeParams& prm, int G, int grid_x, cudaStream_t s) {
+  // Paired launches exist for the 16-bit types (fp32 caches launch one row per CTA).
+  if constexpr (!std::is_same<T, float>::value) {
+    if (prm.pair_from > 0) {
+      switch (G) {
+        case 1: return launch_decode<T, D, 1, false, true>(prm, grid_x, s);
+        case 2: return launch_decode<T, D, 2, false, true>(prm, grid_x, s);
+        case 4: return launch_decode<T, D, 4, false, true>(prm, grid_x, s);
+        case 8: return launch_decode<T, D, 8, false, true>(prm, grid_x, s);
+      }
+      return PA_ERR_UNSUPPORTED;
+    }
+  }
+  DecodeParams one = prm;
+  one.pair_from = 0;
   switch (G) {
-    case 1: return launch_decode<T, D, 1>(prm, grid_x, s);
-    case 2: return launch_decode<T, D, 2>(prm, grid_x, s);
-    case 4: return launch_decode<T, D, 4>(prm, grid_x, s);
-    case 8: return launch_decode<T, D, 8>(prm, grid_x, s);
+    case 1: return launch_decode<T, D, 1>(one, grid_x, s);
+    case 2: return launch_decode<T, D, 2>(one, grid_x, s);
+    case 4: return launch_decode<T, D, 4>(one, grid_x, s);
+    case 8: return launch_decode<T, D, 8>(one, grid_x, s);
   }
   return PA_ERR_UNSUPPORTED;
 }
