@@ -117,6 +117,22 @@ def workload_bytes(batch):
                 attend_logical=kv_logical + q_out + tables, attend_unique=kv_unique + q_out + tables)
 
 
+
+def workload_config(name, batch_cpu, partition_arg, world):
+    """The line's `config`: the workload and its sizes only, the same for both arms (the reference arm
+    builds it from the same batch without loading the library); how a step runs it is in `step_plan`."""
+    acct = workload_bytes(batch_cpu)
+    cascade = name == "chat_trace" and partition_arg == "auto"
+    return {
+        "workload": WORKLOAD_DESC[name], "num_seqs": batch_cpu.num_seqs, "block_size": batch_cpu.block_size,
+        "head_dim": batch_cpu.head_dim, "num_q_heads": batch_cpu.num_q_heads,
+        "num_kv_heads": batch_cpu.num_kv_heads,
+        "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush" if not cascade else
+              "unique KV (522 MB) larger than L2, no flush; the shared prefix is read once per step by design",
+        "kv_bytes_logical_per_rank": acct["kv_logical"], "kv_bytes_unique_per_rank": acct["kv_unique"],
+        "parallelism": f"dp{world} (independent batches per GPU)",
+    }
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -450,7 +466,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": WORKLOAD_DESC[args.workload], "block_size": args.block_size},
+        "data": "synthetic", "config": workload_config(args.workload, batch, args.partition, args.gpus),
         "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
                          "cpu_model": cpu_model(), "cpu_count": os.cpu_count(),
                          "sample": f"first {n} of {batch.num_seqs} sequences per step, fp64 numpy"},
@@ -733,16 +749,9 @@ def measure(name, block_size, partition_arg, K, W, rank, world, sampler, do_e2e=
     res = {
         "value": value, "unit": unit, "ms_per_step": ms_step, "steps": n_long if long_timed else K, "warmup": W,
         "dtype": batch_cpu.info["dtype"],
-        "config": {
-            "workload": WORKLOAD_DESC[name], "num_seqs": batch.num_seqs, "block_size": batch.block_size,
-            "head_dim": batch.head_dim, "num_q_heads": batch.num_q_heads, "num_kv_heads": batch.num_kv_heads,
-            "partition": partition, "fused_append": fused,
-            "shared_prefix": list(step.shared_prefix) if cascade else None,
-            "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush" if not cascade else
-                  "unique KV (522 MB) larger than L2, no flush; the shared prefix is read once per step by design",
-            "kv_bytes_logical_per_rank": acct["kv_logical"], "kv_bytes_unique_per_rank": acct["kv_unique"],
-            "parallelism": f"dp{world} (independent batches per GPU)",
-        },
+        "config": workload_config(name, batch_cpu, partition_arg if not prefill else "auto", world),
+        "step_plan": {"partition": partition, "fused_append": fused,
+                      "shared_prefix": list(step.shared_prefix) if cascade else None},
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": step.launches_per_call * (n_long if long_timed else K),
@@ -909,6 +918,7 @@ def run_ours(args):
             "metric": METRIC, "value": main["value"], "unit": main["unit"], "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": main["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": main["dtype"], "data": "synthetic", "config": main["config"],
+            "step_plan": main["step_plan"],
             "roofline": main["roofline"], "cpu_baseline": main.get("cpu_baseline"), "e2e": main["e2e"],
             "gpu_launches": main["gpu_launches"],
             "clocks": main["clocks"], "sustained": main["sustained"],

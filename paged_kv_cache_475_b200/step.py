@@ -44,8 +44,9 @@ class DecodeStep:
 
     shared_prefix=(prefix_len, group_size): sequences 0..group_size-1 share the
     blocks of their first prefix_len tokens; the step then runs the cascade of
-    pa_decode_shared_prefix (prefix once per group on the tensor cores, the
-    rest split-KV, merge), with the newest tokens' K/V written on the way.
+    pa_decode_shared_prefix (prefix once per group on the tensor cores, every
+    sequence's own tokens in one decode pass, then the merge of the group's
+    rows), with the newest tokens' K/V written on the way.
     """
 
     def __init__(self, num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
