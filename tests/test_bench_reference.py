@@ -35,3 +35,17 @@ def test_reference_other_ranks_exit_quietly():
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
 
+
+
+def test_reference_config_is_the_workload_config_of_our_arm():
+    """Both arms describe the same workload: the reference line's config is what our arm's line carries
+    for the same workload and arguments (the bounded sample is named in cpu_baseline.sample)."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    r = _run(0, "--gpus", "2")
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    ours = bench.workload_config("llama_decode", bench.make_workload("llama_decode", 16), "auto", 2)
+    assert line["config"] == ours
+    assert "sequences per step" in line["cpu_baseline"]["sample"]
