@@ -62,6 +62,15 @@ constexpr int kN = 64;         // keys per tile
 #endif
 constexpr int kStagesK = PA_TC_KSTAGES;  // K ring (16 KB per stage at D = 128)
 constexpr int kStagesV = PA_TC_VSTAGES;  // V ring
+#ifndef PA_TC_SLOT_BY_COMPLETION
+// With two-slot rings a K slot is free once the S two tiles back has
+// completed, and a V slot once the PV two tiles back has: the producers wait
+// on those barriers (s_full / o_done), so the MMA thread issues no commit of
+// its own to release a slot.
+#define PA_TC_SLOT_BY_COMPLETION 1
+#endif
+static_assert(!PA_TC_SLOT_BY_COMPLETION || (kStagesK == 2 && kStagesV == 2),
+              "slot release through s_full / o_done needs two-slot rings");
 #ifndef PA_TC_BT_STAGED
 #define PA_TC_BT_STAGED 0  // block-table entries staged in shared memory (0: each read one tile ahead; 128 / 256 / 1024 measured 1 / 2 / 3% slower)
 #endif
@@ -480,7 +489,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const int stages = is_k ? kStagesK : kStagesV;
       int n_tiles_local = n_tiles;
       uint64_t* full = is_k ? k_full : v_full;
+#if !PA_TC_SLOT_BY_COMPLETION
       uint64_t* empty = is_k ? k_empty : v_empty;
+#endif
       const CUtensorMap* map = is_k ? &tm_k : &tm_v;
       const uint32_t ring = is_k ? sK : sV;
       // The CTA's pages [jb0, jb0 + n_bt) as TMA row coordinates, staged
@@ -526,7 +537,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int st = j % stages;
         const int y = y_next;
         y_next = row_of(j + 1);  // issued before the wait, so a global lookup's latency hides behind it
+#if PA_TC_SLOT_BY_COMPLETION
+        // slot st last held tile j - 2: free once S(j - 2) (K) or PV(j - 2) (V)
+        // has completed, phase (j - 2) / 2 of that tile's buffer barrier
+        if (j >= 2 && !wait_all(is_k ? &s_full[j & 1] : &o_done[j & 1], ((j - 2) >> 1) & 1)) {
+#else
         if (!wait_all(&empty[st], ((j / stages) & 1) ^ 1)) {
+#endif
           if (lane == 0) set_error(p.err, PA_DEVERR_WAIT);
           break;
         }
@@ -572,7 +589,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           tc_mma_ts(tO, tP + kk * 8, bd, kIdescO, (k > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(&o_done[k & 1]);
+#if !PA_TC_SLOT_BY_COMPLETION
         tc_commit(&v_empty[st]);
+#endif
       }
       __syncwarp();
       PA_TR(kEvMmaPVIssued, k);
@@ -595,7 +614,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           tc_mma(tS, ad, bd, kIdescS, ks > 0 ? 1u : 0u);
         }
         tc_commit(&s_full[j & 1]);
+#if !PA_TC_SLOT_BY_COMPLETION
         tc_commit(&k_empty[st]);
+#endif
       }
       __syncwarp();
       PA_TR(kEvMmaSIssued, j);
