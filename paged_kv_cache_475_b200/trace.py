@@ -77,7 +77,9 @@ def summarize_prefill(rec):
         ok = idx < n
         y = np.full(x.shape, np.nan)
         y[ok] = E[b][idx[ok]]
-        return float(np.nanmean(y - x))
+        d = y - x
+        # events this build does not record are NaN throughout: report NaN without a warning
+        return float(np.nanmean(d)) if np.isfinite(d).any() else float("nan")
 
     period = np.diff(E["mma_s_issued"])
     return {
